@@ -1,0 +1,133 @@
+"""Oracle: choosing the query-key tile pairs that run in BF16.
+
+TEST INFRASTRUCTURE (see ``oracle/formats.py``): only tests, the smoke check
+and the benchmark's CPU-baseline leg use this module.
+
+What it follows.  ThriftAttention: Selective Mixed Precision for
+Long-Context FP4 Attention (abstract, first stage): a cheap heuristic picks
+a small number of important query-key block pairs for high precision.
+HyQuant: Hybrid-Precision Quantization for LLM Attention (abstract) keeps
+vertical-line (sink) tokens and the local window in high precision.  The
+pages do not give the heuristic, so this library fixes it:
+
+1. pool: per 128-row tile t and channel c, the mean of the original BF16
+   values over the tile's valid rows, summed in FP32 in ascending row order
+   and divided by the row count;
+2. score(i, j) = sum_c qp[h][i][c] * kp[h/G][j][c], FP32 products and FP32
+   additions in ascending c, starting from +0 (no fused multiply-add);
+3. candidates C_i = {0..i} (causal) or {0..T-1}; forced F_i = {0, i} & C_i
+   (sink tile and diagonal / local window);
+4. budget k_i: ``budget_tiles > 0`` -> min(n_i, max(|F_i|, budget_tiles));
+   else bp = budget_bp: 0 -> 0 (no forced tiles either), >= 10000 -> n_i,
+   otherwise min(n_i, max(|F_i|, ceil(bp * n_i / 10000)));
+5. the forced tiles (when k_i > 0) plus the k_i - |F_i| best remaining
+   candidates by (score descending, index ascending; -0 equals +0).
+
+The result is a bitmask ``mask[B,Hq,T,ceil(T/32)]`` of uint32 words: bit
+j % 32 of word j // 32 set means tile pair (i, j) runs in BF16.
+
+Parity pins: tests/test_oracle_select.py (planted scores recover the planted
+tiles, top-k dominance, popcounts, causal emptiness, budget extremes,
+nesting of budgets, pooled means against float64 means).
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+F32 = np.float32
+
+
+def _as_f32(x) -> np.ndarray:
+    if isinstance(x, torch.Tensor):
+        return x.detach().to("cpu", torch.float32).numpy()
+    return np.asarray(x, dtype=np.float32)
+
+
+def pool_tiles(x) -> np.ndarray:
+    """x[B,H,N,d] -> per-tile column means [B,H,T,d] (FP32, ascending row sums)."""
+    x = _as_f32(x)
+    B, H, N, d = x.shape
+    T = (N + 127) // 128
+    out = np.zeros((B, H, T, d), dtype=F32)
+    for t in range(T):
+        r0 = t * 128
+        cnt = min(128, N - r0)
+        acc = np.zeros((B, H, d), dtype=F32)
+        for r in range(cnt):
+            acc = (acc + x[:, :, r0 + r, :]).astype(F32)
+        out[:, :, t, :] = (acc / F32(cnt)).astype(F32)
+    return out
+
+
+def tile_scores(qp, kp, Hq: int, Hkv: int) -> np.ndarray:
+    """scores[B,Hq,T,T] = FP32 dot products of pooled means, ascending c."""
+    qp = np.asarray(qp, dtype=F32)
+    kp = np.asarray(kp, dtype=F32)
+    G = Hq // Hkv
+    kp_q = np.repeat(kp, G, axis=1)                  # query head h uses kv head h // G
+    B, H, T, d = qp.shape
+    acc = np.zeros((B, H, T, T), dtype=F32)
+    for c in range(d):
+        prod = (qp[:, :, :, None, c] * kp_q[:, :, None, :, c]).astype(F32)
+        acc = (acc + prod).astype(F32)
+    return acc
+
+
+def budget_for_row(n_i: int, n_forced: int, budget_bp: int, budget_tiles: int) -> int:
+    if budget_tiles > 0:
+        return min(n_i, max(n_forced, budget_tiles))
+    if budget_bp <= 0:
+        return 0
+    if budget_bp >= 10000:
+        return n_i
+    want = (budget_bp * n_i + 9999) // 10000
+    return min(n_i, max(n_forced, want))
+
+
+def select_rows(scores, causal: bool, budget_bp: int, budget_tiles: int):
+    """scores[B,Hq,T,T] -> (mask[B,Hq,T,W] uint32, counts[B,Hq,T] int32)."""
+    scores = np.asarray(scores, dtype=F32)
+    B, H, T, _ = scores.shape
+    W = (T + 31) // 32
+    mask = np.zeros((B, H, T, W), dtype=np.uint32)
+    counts = np.zeros((B, H, T), dtype=np.int32)
+    for b in range(B):
+        for h in range(H):
+            for i in range(T):
+                n_i = i + 1 if causal else T
+                forced = sorted({0, i} & set(range(n_i)))
+                k_i = budget_for_row(n_i, len(forced), budget_bp, budget_tiles)
+                chosen = []
+                if k_i > 0:
+                    chosen = list(forced)
+                    rest = [j for j in range(n_i) if j not in forced]
+                    s = scores[b, h, i, rest].astype(np.float64)   # -0 == +0 in comparisons
+                    order = np.lexsort((np.asarray(rest), -s))     # score desc, then index asc
+                    chosen += [rest[o] for o in order[: k_i - len(forced)]]
+                for j in chosen:
+                    mask[b, h, i, j // 32] |= np.uint32(1) << np.uint32(j % 32)
+                counts[b, h, i] = len(chosen)
+    return mask, counts
+
+
+def select(q, k, causal: bool, budget_bp: int, budget_tiles: int = 0):
+    """The library's ``thrift_select``: pooled scores -> BF16 tile mask."""
+    qp = pool_tiles(q)
+    kp = pool_tiles(k)
+    Hq, Hkv = qp.shape[1], kp.shape[1]
+    sc = tile_scores(qp, kp, Hq, Hkv)
+    mask, counts = select_rows(sc, causal, budget_bp, budget_tiles)
+    return dict(qp=qp, kp=kp, scores=sc, mask=mask, counts=counts)
+
+
+def mask_bit(mask, b: int, h: int, i: int, j: int) -> bool:
+    return bool((int(mask[b, h, i, j // 32]) >> (j % 32)) & 1)
+
+
+def mask_to_dense(mask, T: int) -> np.ndarray:
+    """[B,H,T,W] words -> [B,H,T,T] bool."""
+    m = np.asarray(mask, dtype=np.uint32)
+    B, H, Tq, W = m.shape
+    bits = ((m[..., :, None] >> np.arange(32, dtype=np.uint32)) & 1).astype(bool)
+    return bits.reshape(B, H, Tq, W * 32)[..., :T]
