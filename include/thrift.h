@@ -1,0 +1,181 @@
+/*
+ * thrift.h -- C ABI of libthrift: mixed FP4/BF16 attention forward (prefill)
+ * for NVIDIA B200 (sm_100a).
+ *
+ * The method.  ThriftAttention: Selective Mixed Precision for Long-Context
+ * FP4 Attention (abstract) runs attention in two stages: a cheap heuristic
+ * picks a few important query-key block pairs for high precision, then the
+ * selected blocks are computed in high precision and all others in 4-bit,
+ * both merged by online softmax into one output.  HyQuant: Hybrid-Precision
+ * Quantization for LLM Attention (abstract) keeps sink ("vertical line")
+ * tokens and the local window in full precision.  Here the high precision
+ * is BF16 (the inputs' own type), the low precision is NVFP4 for Q and K
+ * and FP8 e4m3 for V and for the probabilities, tiles are 128 x 128.
+ *
+ * Three calls make one forward pass, in this order, on one stream:
+ *   thrift_quantize  -> NVFP4 Q, K and FP8 V            (stage 0: operands)
+ *   thrift_select    -> bitmask of BF16 tile pairs       (stage 1)
+ *   thrift_attn_fwd  -> O (and optionally LSE)           (stage 2)
+ *
+ * Conventions for every call:
+ *  - All tensor arguments are DEVICE pointers, allocated and owned by the
+ *    caller; the library allocates no device memory.  Inputs are BF16,
+ *    contiguous, head-major: q[B][Hq][N][d], k and v [B][Hkv][N][d].
+ *    Every pointer must be 16-byte aligned.
+ *  - Query head h reads key/value head h / (Hq / Hkv).
+ *  - All work is enqueued on `stream` (a cudaStream_t, 0 = legacy default);
+ *    no call synchronises.  Host-side argument errors are returned before
+ *    anything is enqueued.  No exception crosses this interface.
+ *  - T = ceil(N / 128) tiles, W = ceil(T / 32) mask words per query tile,
+ *    Np = 128 * T (N padded to whole tiles).
+ *  - Inputs must be finite; non-finite values give undefined results.
+ *  - Supported: d in {64, 128}; Hq % Hkv == 0; 1 <= N; causal in {0, 1}.
+ */
+#ifndef THRIFT_H
+#define THRIFT_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define THRIFT_API __attribute__((visibility("default")))
+#else
+#define THRIFT_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  THRIFT_OK = 0,
+  THRIFT_ERR_INVALID = 1,      /* bad argument (null / misaligned pointer, bad size) */
+  THRIFT_ERR_UNSUPPORTED = 2,  /* valid but not supported (e.g. d not in {64,128}) */
+  THRIFT_ERR_CUDA = 3,         /* a CUDA runtime/driver call failed */
+  THRIFT_ERR_TIMEOUT = 4       /* a kernel's bounded wait gave up (device watchdog) */
+} thrift_status;
+
+/* Problem shape.  softmax_scale == 0 selects 1/sqrt(d). */
+typedef struct {
+  int32_t B, Hq, Hkv, N, d;
+  int32_t causal;
+  float softmax_scale;
+} thrift_shape;
+
+/*
+ * Quantised operands written by thrift_quantize and read by thrift_attn_fwd.
+ * Device pointers, caller-owned; sizes from thrift_quant_bytes().
+ *
+ * NVFP4 (Q and K): per (batch, head) tensor scale g = amax / 2688 (1 for an
+ * all-zero head); per 16 consecutive elements along d an e4m3 scale
+ * s = e4m3(amax_blk / (6 g)); element code e2m1(x / (dec(s) g)); all
+ * arithmetic in FP32 with correctly rounded operations, round-to-nearest-even,
+ * saturating; a block whose scale decodes to 0 gets zero codes.
+ *
+ * FP8 V: per (batch, kv head, channel c) the smallest integer e_c with
+ * amax_c <= 448 * 2^e_c (0 for a zero channel); v_code = e4m3(v * 2^-e_c)
+ * and the exact BF16 copy v * 2^-e_c, both stored transposed (channel-major)
+ * and zero-padded to Np keys.
+ */
+typedef struct {
+  uint8_t *q_fp4;     /* [B][Hq][N][d/2]   e2m1 codes, element 2t in the low nibble */
+  uint8_t *q_sf;      /* [B][Hq][N][d/16]  e4m3 block scales, row-major             */
+  uint8_t *q_sf_mma;  /* [B][Hq][T][d/64][512] the same scales in tensor-core order:
+                         byte r0*16 + r1*4 + k of chunk kb holds the scale of row
+                         128 t + 32 r1 + r0, block 4 kb + k; rows >= N hold 0     */
+  float   *q_gs;      /* [B][Hq]           tensor scales g                          */
+  uint8_t *k_fp4;     /* [B][Hkv][N][d/2]                                           */
+  uint8_t *k_sf;      /* [B][Hkv][N][d/16]                                          */
+  uint8_t *k_sf_mma;  /* [B][Hkv][T][d/64][512]                                     */
+  float   *k_gs;      /* [B][Hkv]                                                   */
+  uint8_t *v_fp8t;    /* [B][Hkv][d][Np]   e4m3 codes of v * 2^-e_c, transposed      */
+  uint16_t *v_st;     /* [B][Hkv][d][Np]   bf16 v * 2^-e_c, transposed               */
+  int8_t  *v_exp;     /* [B][Hkv][d]       e_c                                       */
+} thrift_quant;
+
+/* Field indices for thrift_quant_bytes, in struct order. */
+enum {
+  THRIFT_Q_FP4 = 0, THRIFT_Q_SF, THRIFT_Q_SF_MMA, THRIFT_Q_GS,
+  THRIFT_K_FP4, THRIFT_K_SF, THRIFT_K_SF_MMA, THRIFT_K_GS,
+  THRIFT_V_FP8T, THRIFT_V_ST, THRIFT_V_EXP, THRIFT_QUANT_NFIELDS
+};
+
+/* Operation indices for thrift_workspace_bytes. */
+enum { THRIFT_OP_QUANTIZE = 0, THRIFT_OP_SELECT = 1, THRIFT_OP_ATTN = 2 };
+
+/* Bytes of one thrift_quant field for `shape` (0 for a bad shape or index). */
+THRIFT_API size_t thrift_quant_bytes(const thrift_shape *shape, int field);
+
+/* Bytes of device workspace an operation needs (0 = none; the pointer may be NULL). */
+THRIFT_API size_t thrift_workspace_bytes(const thrift_shape *shape, int op);
+
+/*
+ * Stage 0: quantise Q, K to NVFP4 and V to FP8 (see thrift_quant).
+ * q, k, v: BF16 device inputs.  out: every field must be non-NULL.
+ * ws: device workspace of thrift_workspace_bytes(shape, THRIFT_OP_QUANTIZE)
+ * bytes (per-head and per-channel amax accumulators, cleared by this call).
+ */
+THRIFT_API thrift_status thrift_quantize(const thrift_shape *shape, const void *q, const void *k,
+                              const void *v, const thrift_quant *out, void *ws,
+                              size_t ws_bytes, void *stream);
+
+/*
+ * Stage 1: the BF16 tile-pair bitmask.
+ * For every (b, hq, query tile i): pooled means qp_i, kp_j (FP32 column sums
+ * over the tile's valid rows in ascending order, divided by the row count);
+ * score(i,j) = sum over c ascending of FP32 products qp_i[c] * kp_j[c] with
+ * FP32 additions (no fused multiply-add); candidates j in {0..i} (causal) or
+ * {0..T-1}; the sink tile 0 and the diagonal tile i are forced; the budget
+ * k_i is min(n_i, max(|forced|, budget_tiles)) when budget_tiles > 0, else
+ * 0 for budget_bp == 0, n_i for budget_bp >= 10000, and
+ * min(n_i, max(|forced|, ceil(budget_bp * n_i / 10000))) otherwise; the
+ * forced tiles plus the best remaining candidates by (score descending,
+ * index ascending) fill it.
+ * mask: [B][Hq][T][W] uint32, bit j%32 of word j/32 = pair (i, j) in BF16.
+ * counts: [B][Hq][T] int32 popcounts, or NULL.
+ * ws: thrift_workspace_bytes(shape, THRIFT_OP_SELECT) bytes (pooled means).
+ */
+THRIFT_API thrift_status thrift_select(const thrift_shape *shape, const void *q, const void *k,
+                            int32_t budget_bp, int32_t budget_tiles, uint32_t *mask,
+                            int32_t *counts, void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * Stage 2: the fused mixed-precision attention forward.
+ * For each (b, hq, query tile i) and key tiles j ascending: BF16 pairs use
+ * S = Q K^T * scale on the BF16 inputs; FP4 pairs use the block-scaled NVFP4
+ * product times g_q g_k * scale; causal / ragged entries are -inf; the
+ * running maximum is exact; p = exp(S - m) in FP32; l accumulates uncast p;
+ * P is cast to e4m3 (FP4 pairs, with FP8 V) or BF16 (BF16 pairs, with the
+ * BF16 V copy) after scaling by 2^8, and both products accumulate into one
+ * FP32 output, which is finally scaled by 2^(e_c - 8) / l.
+ * q, k: the BF16 inputs (read on BF16 pairs).  mask from thrift_select.
+ * o: [B][Hq][N][d] BF16 output.  lse: [B][Hq][N] FP32 natural-log
+ * log-sum-exp of the scaled logits, or NULL.
+ * ws: may be NULL (thrift_workspace_bytes(..., THRIFT_OP_ATTN) == 0).
+ */
+THRIFT_API thrift_status thrift_attn_fwd(const thrift_shape *shape, const thrift_quant *quant,
+                              const void *q, const void *k, const uint32_t *mask,
+                              void *o, float *lse, void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * Synchronises `stream`, then reads and clears the library's device error
+ * word.  Returns THRIFT_ERR_TIMEOUT if a kernel's bounded wait gave up since
+ * the last call (the kernel then returned early and its outputs are
+ * undefined); *detail (if non-NULL) receives the raw error word.
+ */
+THRIFT_API thrift_status thrift_device_status(void *stream, uint32_t *detail);
+
+/* Human-readable name of a status code (static storage). */
+THRIFT_API const char *thrift_status_string(thrift_status status);
+
+/* Number of kernels this library has launched since load (all devices). */
+THRIFT_API uint64_t thrift_launch_count(void);
+
+/* Library version string. */
+THRIFT_API const char *thrift_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* THRIFT_H */

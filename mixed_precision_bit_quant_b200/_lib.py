@@ -1,0 +1,208 @@
+"""ctypes binding of libthrift (include/thrift.h): argument marshalling only.
+
+Every step of the path runs in the library's CUDA kernels; this module only
+allocates output tensors with PyTorch, passes device pointers and the
+current stream, and turns status codes into exceptions.  There is no CPU
+fallback: if the library is missing, :func:`lib` raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import dataclasses
+import os
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libthrift.so")
+
+THRIFT_OK, THRIFT_ERR_INVALID, THRIFT_ERR_UNSUPPORTED, THRIFT_ERR_CUDA, THRIFT_ERR_TIMEOUT = range(5)
+OP_QUANTIZE, OP_SELECT, OP_ATTN = range(3)
+QUANT_FIELDS = ["q_fp4", "q_sf", "q_sf_mma", "q_gs", "k_fp4", "k_sf", "k_sf_mma", "k_gs",
+                "v_fp8t", "v_st", "v_exp"]
+_FIELD_DTYPES = {"q_gs": torch.float32, "k_gs": torch.float32, "v_st": torch.bfloat16,
+                 "v_exp": torch.int8}
+
+
+class ThriftError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {status_string(status)}")
+
+
+class Shape(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int32), ("Hq", ctypes.c_int32), ("Hkv", ctypes.c_int32),
+                ("N", ctypes.c_int32), ("d", ctypes.c_int32), ("causal", ctypes.c_int32),
+                ("softmax_scale", ctypes.c_float)]
+
+
+class QuantStruct(ctypes.Structure):
+    _fields_ = [(f, ctypes.c_void_p) for f in QUANT_FIELDS]
+
+
+_lib: Optional[ctypes.CDLL] = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libthrift.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"libthrift.so not found at {LIB_PATH}; build it with "
+                               "`python -m mixed_precision_bit_quant_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        P, S, I32, U64 = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int32, ctypes.c_uint64
+        SP = ctypes.POINTER(Shape)
+        QP = ctypes.POINTER(QuantStruct)
+        L.thrift_quant_bytes.argtypes = [SP, ctypes.c_int]
+        L.thrift_quant_bytes.restype = S
+        L.thrift_workspace_bytes.argtypes = [SP, ctypes.c_int]
+        L.thrift_workspace_bytes.restype = S
+        L.thrift_quantize.argtypes = [SP, P, P, P, QP, P, S, P]
+        L.thrift_quantize.restype = ctypes.c_int
+        L.thrift_select.argtypes = [SP, P, P, I32, I32, P, P, P, S, P]
+        L.thrift_select.restype = ctypes.c_int
+        L.thrift_attn_fwd.argtypes = [SP, QP, P, P, P, P, P, P, S, P]
+        L.thrift_attn_fwd.restype = ctypes.c_int
+        L.thrift_device_status.argtypes = [P, ctypes.POINTER(ctypes.c_uint32)]
+        L.thrift_device_status.restype = ctypes.c_int
+        L.thrift_status_string.argtypes = [ctypes.c_int]
+        L.thrift_status_string.restype = ctypes.c_char_p
+        L.thrift_launch_count.argtypes = []
+        L.thrift_launch_count.restype = U64
+        L.thrift_version.argtypes = []
+        L.thrift_version.restype = ctypes.c_char_p
+        _lib = L
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().thrift_status_string(int(status)).decode()
+
+
+def _check(status: int, what: str) -> None:
+    if status != THRIFT_OK:
+        raise ThriftError(status, what)
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _stream() -> int:
+    return torch.cuda.current_stream().cuda_stream
+
+
+def make_shape(B, Hq, Hkv, N, d, causal, softmax_scale: float = 0.0) -> Shape:
+    return Shape(int(B), int(Hq), int(Hkv), int(N), int(d), int(bool(causal)), float(softmax_scale))
+
+
+def shape_of(q: torch.Tensor, k: torch.Tensor, causal: bool, softmax_scale: float = 0.0) -> Shape:
+    B, Hq, N, d = q.shape
+    return make_shape(B, Hq, k.shape[1], N, d, causal, softmax_scale)
+
+
+def quant_bytes(shape: Shape, field: int) -> int:
+    return int(lib().thrift_quant_bytes(ctypes.byref(shape), field))
+
+
+def workspace_bytes(shape: Shape, op: int) -> int:
+    return int(lib().thrift_workspace_bytes(ctypes.byref(shape), op))
+
+
+@dataclasses.dataclass
+class Quantized:
+    """The quantised operands (device tensors), in thrift_quant field order."""
+    tensors: dict
+
+    def struct(self) -> QuantStruct:
+        return QuantStruct(*[self.tensors[f].data_ptr() for f in QUANT_FIELDS])
+
+    def __getitem__(self, k):
+        return self.tensors[k]
+
+
+def alloc_quantized(shape: Shape, device) -> Quantized:
+    out = {}
+    for idx, f in enumerate(QUANT_FIELDS):
+        nbytes = quant_bytes(shape, idx)
+        if nbytes == 0:
+            raise ThriftError(THRIFT_ERR_INVALID, "thrift_quant_bytes")
+        dt = _FIELD_DTYPES.get(f, torch.uint8)
+        out[f] = torch.empty(nbytes // torch.empty((), dtype=dt).element_size(), dtype=dt, device=device)
+    return Quantized(out)
+
+
+def _workspace(shape: Shape, op: int, device) -> Optional[torch.Tensor]:
+    n = workspace_bytes(shape, op)
+    return torch.empty(max(n, 16), dtype=torch.uint8, device=device) if n > 0 else None
+
+
+def quantize(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = False,
+             out: Optional[Quantized] = None, ws: Optional[torch.Tensor] = None) -> Quantized:
+    """thrift_quantize: NVFP4 Q, K and FP8 V (all device tensors)."""
+    shape = shape_of(q, k, causal)
+    out = out if out is not None else alloc_quantized(shape, q.device)
+    ws = ws if ws is not None else _workspace(shape, OP_QUANTIZE, q.device)
+    st = out.struct()
+    _check(lib().thrift_quantize(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), ctypes.byref(st),
+                                 _ptr(ws), 0 if ws is None else ws.numel(), _stream()), "thrift_quantize")
+    return out
+
+
+def select(q: torch.Tensor, k: torch.Tensor, causal: bool, budget_bp: int = 500, budget_tiles: int = 0,
+           mask: Optional[torch.Tensor] = None, counts: Optional[torch.Tensor] = None,
+           ws: Optional[torch.Tensor] = None):
+    """thrift_select: returns (mask[B,Hq,T,W] int32 view of the uint32 words, counts[B,Hq,T])."""
+    shape = shape_of(q, k, causal)
+    B, Hq, N, _ = q.shape
+    T = (N + 127) // 128
+    W = (T + 31) // 32
+    if mask is None:
+        mask = torch.empty((B, Hq, T, W), dtype=torch.int32, device=q.device)
+    if counts is None:
+        counts = torch.empty((B, Hq, T), dtype=torch.int32, device=q.device)
+    ws = ws if ws is not None else _workspace(shape, OP_SELECT, q.device)
+    _check(lib().thrift_select(ctypes.byref(shape), _ptr(q), _ptr(k), int(budget_bp), int(budget_tiles),
+                               _ptr(mask), _ptr(counts), _ptr(ws), 0 if ws is None else ws.numel(),
+                               _stream()), "thrift_select")
+    return mask, counts
+
+
+def attn_fwd(q: torch.Tensor, k: torch.Tensor, quant: Quantized, mask: torch.Tensor, causal: bool,
+             softmax_scale: float = 0.0, o: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+             want_lse: bool = False):
+    """thrift_attn_fwd: returns (o[B,Hq,N,d] bf16, lse[B,Hq,N] fp32 or None)."""
+    shape = shape_of(q, k, causal, softmax_scale)
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty(q.shape[:3], dtype=torch.float32, device=q.device)
+    st = quant.struct()
+    _check(lib().thrift_attn_fwd(ctypes.byref(shape), ctypes.byref(st), _ptr(q), _ptr(k), _ptr(mask),
+                                 _ptr(o), _ptr(lse), None, 0, _stream()), "thrift_attn_fwd")
+    return o, lse
+
+
+def attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool, budget_bp: int = 500,
+              budget_tiles: int = 0, softmax_scale: float = 0.0, want_lse: bool = False):
+    """The whole forward pass: quantize -> select -> fused mixed attention."""
+    quant = quantize(q, k, v, causal)
+    mask, _ = select(q, k, causal, budget_bp, budget_tiles)
+    return attn_fwd(q, k, quant, mask, causal, softmax_scale, want_lse=want_lse)
+
+
+def device_status() -> tuple:
+    """Synchronise the current stream and read (status, raw word) of the device watchdog."""
+    w = ctypes.c_uint32(0)
+    s = lib().thrift_device_status(_stream(), ctypes.byref(w))
+    return int(s), int(w.value)
+
+
+def launch_count() -> int:
+    return int(lib().thrift_launch_count())
+
+
+def version() -> str:
+    return lib().thrift_version().decode()

@@ -1,0 +1,487 @@
+// Stage 2: fused mixed FP4 / BF16 attention forward on tcgen05 tensor cores.
+//
+// ThriftAttention: Selective Mixed Precision for Long-Context FP4 Attention
+// (abstract, second stage): the selected query-key blocks are computed in
+// high precision and the rest in FP4, both merged by online softmax into a
+// single output.  HyQuant: Hybrid-Precision Quantization for LLM Attention
+// (abstract): one hybrid-precision attention operator for prefill.
+//
+// One CTA computes one 128-row query tile (b, hq, i) against the key tiles
+// j = 0 .. (causal ? i : T-1) in ascending order.  Warp roles:
+//   warps 0-3  softmax: one thread per query row (= TMEM lane); reads S from
+//              TMEM, masks, exact running max, exp2, row sums, writes P back
+//              into TMEM (e4m3 or bf16), rescales O in TMEM when the row max
+//              grows, final epilogue O * 2^e_c / l -> bf16.
+//   warp 4     TMA producer: Q (NVFP4 + scales + BF16) once, then per key
+//              tile either NVFP4 K + scales and e4m3 V^T, or BF16 K and V^T,
+//              following the tile's mask bit; two stages each.
+//   warp 5     TMEM allocator and MMA issuer (one thread):
+//              FP4 pair: S = Q4 K4^T  kind::mxf4nvf4 (block scales in TMEM)
+//                        O += P8 V8   kind::f8f6f4, P read from TMEM
+//              BF16 pair: S = Q K^T   kind::f16
+//                        O += P16 Vs  kind::f16, P read from TMEM
+// TMEM columns: S double buffer [0,256), O [256, 256+D), scale factors after.
+// The S computation of tile j+1 overlaps the softmax of tile j.
+#include <cuda.h>
+
+#include "dev.cuh"
+#include "kernels.h"
+
+namespace thrift {
+
+__device__ uint32_t g_attn_error_word;
+
+namespace attn {
+
+constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s per wait: far above any legitimate wait
+constexpr int kThreads = 192;
+constexpr int kMaxW = 128;                          // mask words per query tile (T <= 4096)
+
+enum Bar : int {
+  Q_FULL = 0, K_FULL = 1, K_EMPTY = 3, V_FULL = 5, V_EMPTY = 7, S_FULL = 9, P_FULL = 11,
+  PV_DONE = 13, O_FINAL = 14, DRAIN = 15, NBAR = 16
+};
+
+__host__ __device__ constexpr int al(int x, int a) { return (x + a - 1) / a * a; }
+
+template <int D>
+struct Layout {
+  static constexpr int QFP4 = 128 * D / 2;    // packed e2m1 Q tile
+  static constexpr int QBF = 128 * D * 2;      // bf16 Q tile (D/64 boxes of 128 x 64)
+  static constexpr int SF = (D / 64) * 512;    // block scales of one tile, tensor-core order
+  static constexpr int KBUF = 128 * D * 2;     // max(e2m1 K tile, bf16 K tile)
+  static constexpr int VBUF = D * 128 * 2;     // max(e4m3 V^T tile, bf16 V^T tile)
+  static constexpr int OFF_QFP4 = 0;
+  static constexpr int OFF_QBF = al(OFF_QFP4 + QFP4, 1024);
+  static constexpr int OFF_K = OFF_QBF + QBF;          // two stages
+  static constexpr int OFF_V = OFF_K + 2 * KBUF;       // two stages
+  static constexpr int OFF_QSF = OFF_V + 2 * VBUF;
+  static constexpr int OFF_KSF = OFF_QSF + SF;         // two stages
+  static constexpr int OFF_BAR = al(OFF_KSF + 2 * SF, 64);
+  static constexpr int OFF_MISC = OFF_BAR + 8 * NBAR;  // tmem holder, abort flag
+  static constexpr int OFF_MASK = OFF_MISC + 16;
+  static constexpr int OFF_VSC = OFF_MASK + 4 * kMaxW;  // per-channel output scales
+  static constexpr int BYTES = OFF_VSC + 4 * D;
+  // request at least 116 KB so that one CTA (and its 512 TMEM columns) owns an SM
+  static constexpr int DYN = (BYTES + 1024 > 116 * 1024) ? BYTES + 1024 : 116 * 1024;
+  // TMEM columns
+  static constexpr uint32_t S_COL0 = 0, O_COL = 256, SFA_COL = 256 + D, SFB_COL0 = SFA_COL + 8;
+};
+
+struct Params {
+  const uint8_t* q_sf_mma;
+  const uint8_t* k_sf_mma;
+  const float* q_gs;
+  const float* k_gs;
+  const int8_t* v_exp;
+  const uint32_t* mask;
+  __nv_bfloat16* o;
+  float* lse;
+  int B, Hq, Hkv, N, T, W, causal;
+  float scale_log2;  // softmax scale * log2(e)
+};
+
+__device__ __forceinline__ void raise_error(volatile int* abort, uint32_t code) {
+  *abort = 1;
+  atomicOr(&g_attn_error_word, code);
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_qfp4, const __grid_constant__ CUtensorMap tm_kfp4,
+                    const __grid_constant__ CUtensorMap tm_qbf, const __grid_constant__ CUtensorMap tm_kbf,
+                    const __grid_constant__ CUtensorMap tm_vfp8, const __grid_constant__ CUtensorMap tm_vbf,
+                    const Params p) {
+  using L = Layout<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sb = smem_u32(smem);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+  // longest rows first for causal problems
+  const int BHq = p.B * p.Hq;
+  const int lin = blockIdx.x;
+  const int i = p.causal ? (p.T - 1 - lin / BHq) : (lin / BHq);
+  const int bhq = lin % BHq;
+  const int b = bhq / p.Hq, h = bhq % p.Hq;
+  const int bhk = b * p.Hkv + h / (p.Hq / p.Hkv);
+  const int nj = p.causal ? i + 1 : p.T;
+
+  auto BAR = [&](int k) -> uint32_t { return sb + L::OFF_BAR + 8 * k; };
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L::OFF_MISC);
+  volatile int* abort = reinterpret_cast<volatile int*>(smem + L::OFF_MISC + 4);
+  uint32_t* mrow = reinterpret_cast<uint32_t*>(smem + L::OFF_MASK);
+  float* vsc = reinterpret_cast<float*>(smem + L::OFF_VSC);
+
+  if (tid == 0) {
+    for (int k = 0; k < NBAR; ++k) mbar_init(BAR(k), (k == P_FULL || k == P_FULL + 1) ? 4 : 1);
+    *abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 5) {
+    tmem_alloc(smem_u32(tmem_holder), 512);
+    tmem_relinquish();
+  }
+  for (int w = tid; w < p.W; w += kThreads) mrow[w] = p.mask[((size_t)bhq * p.T + i) * p.W + w];
+  for (int c = tid; c < D; c += kThreads) vsc[c] = pow2f((int)p.v_exp[(size_t)bhk * D + c]);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+  auto is_hi = [&](int j) -> bool { return (mrow[j >> 5] >> (j & 31)) & 1u; };
+  volatile int never = 0;
+
+  if (warp == 4) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      prefetch_tmap(&tm_qfp4); prefetch_tmap(&tm_kfp4); prefetch_tmap(&tm_qbf);
+      prefetch_tmap(&tm_kbf); prefetch_tmap(&tm_vfp8); prefetch_tmap(&tm_vbf);
+      mbar_expect_tx(BAR(Q_FULL), L::QFP4 + L::QBF + L::SF);
+      tma_load_3d(sb + L::OFF_QFP4, &tm_qfp4, 0, i * 128, bhq, BAR(Q_FULL));
+      tma_load_3d(sb + L::OFF_QBF, &tm_qbf, 0, i * 128, bhq, BAR(Q_FULL));
+      if (D == 128) tma_load_3d(sb + L::OFF_QBF + 16384, &tm_qbf, 64, i * 128, bhq, BAR(Q_FULL));
+      bulk_load(sb + L::OFF_QSF, p.q_sf_mma + ((size_t)bhq * p.T + i) * L::SF, L::SF, BAR(Q_FULL));
+      int fills[2] = {0, 0};
+      for (int j = 0; j < nj; ++j) {
+        const int s = j & 1, u = j >> 1;
+        const bool hi = is_hi(j);
+        const uint32_t kb = sb + L::OFF_K + s * L::KBUF;
+        const uint32_t vb = sb + L::OFF_V + s * L::VBUF;
+        if (u > 0 && !mbar_wait(BAR(K_EMPTY + s), (u - 1) & 1, abort, kWaitLimitNs)) { raise_error(abort, 1u); break; }
+        if (hi) {
+          mbar_expect_tx(BAR(K_FULL + s), 128 * D * 2);
+          tma_load_3d(kb, &tm_kbf, 0, j * 128, bhk, BAR(K_FULL + s));
+          if (D == 128) tma_load_3d(kb + 16384, &tm_kbf, 64, j * 128, bhk, BAR(K_FULL + s));
+        } else {
+          mbar_expect_tx(BAR(K_FULL + s), L::QFP4 + L::SF);
+          tma_load_3d(kb, &tm_kfp4, 0, j * 128, bhk, BAR(K_FULL + s));
+          bulk_load(sb + L::OFF_KSF + s * L::SF, p.k_sf_mma + ((size_t)bhk * p.T + j) * L::SF, L::SF,
+                    BAR(K_FULL + s));
+        }
+        if (u > 0 && !mbar_wait(BAR(V_EMPTY + s), (u - 1) & 1, abort, kWaitLimitNs)) { raise_error(abort, 1u); break; }
+        if (hi) {
+          mbar_expect_tx(BAR(V_FULL + s), D * 128 * 2);
+          tma_load_3d(vb, &tm_vbf, j * 128, 0, bhk, BAR(V_FULL + s));
+          tma_load_3d(vb + D * 128, &tm_vbf, j * 128 + 64, 0, bhk, BAR(V_FULL + s));
+        } else {
+          mbar_expect_tx(BAR(V_FULL + s), D * 128);
+          tma_load_3d(vb, &tm_vfp8, j * 128, 0, bhk, BAR(V_FULL + s));
+        }
+        fills[s] = u + 1;
+      }
+      if (*abort) {
+        // let copies already in flight land before the CTA's shared memory goes away
+        mbar_wait(BAR(Q_FULL), 0, &never, kWaitLimitNs / 4);
+        for (int s = 0; s < 2; ++s)
+          if (fills[s] > 0) {
+            mbar_wait(BAR(K_FULL + s), (fills[s] - 1) & 1, &never, kWaitLimitNs / 4);
+            mbar_wait(BAR(V_FULL + s), (fills[s] - 1) & 1, &never, kWaitLimitNs / 4);
+          }
+      }
+    }
+  } else if (warp == 5) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr int KB = D / 64;
+      constexpr uint32_t fp4_row = D / 2;
+      constexpr uint32_t fp4_swz = (D == 128) ? SWZ_64B : SWZ_32B;
+      bool ok = mbar_wait(BAR(Q_FULL), 0, abort, kWaitLimitNs);
+      if (!ok) raise_error(abort, 2u);
+      if (ok) {
+        tc_fence_after();
+#pragma unroll
+        for (int kb = 0; kb < KB; ++kb)
+          tmem_cp_32x128b_x4(tmem + L::SFA_COL + 4 * kb, smem_desc(sb + L::OFF_QSF + kb * 512, 16, 128, SWZ_NONE));
+      }
+      for (int j = 0; ok && j <= nj; ++j) {
+        if (j < nj) {
+          const int s = j & 1, u = j >> 1;
+          if (!mbar_wait(BAR(K_FULL + s), u & 1, abort, kWaitLimitNs)) { raise_error(abort, 2u); ok = false; break; }
+          tc_fence_after();
+          const uint32_t d_s = tmem + L::S_COL0 + 128 * s;
+          const uint32_t kb_addr = sb + L::OFF_K + s * L::KBUF;
+          if (is_hi(j)) {
+#pragma unroll
+            for (int k = 0; k < D / 16; ++k) {
+              const uint32_t off = (k >> 2) * 16384 + (k & 3) * 32;
+              mma_bf16_ss(d_s, smem_desc(sb + L::OFF_QBF + off, 16, 1024, SWZ_128B),
+                          smem_desc(kb_addr + off, 16, 1024, SWZ_128B), idesc_bf16(128), k > 0);
+            }
+          } else {
+            const uint32_t sfb = tmem + L::SFB_COL0 + 8 * s;
+#pragma unroll
+            for (int kb = 0; kb < KB; ++kb)
+              tmem_cp_32x128b_x4(sfb + 4 * kb, smem_desc(sb + L::OFF_KSF + s * L::SF + kb * 512, 16, 128, SWZ_NONE));
+#pragma unroll
+            for (int kb = 0; kb < KB; ++kb)
+              mma_nvfp4_ss(d_s, smem_desc(sb + L::OFF_QFP4 + kb * 32, 16, 8 * fp4_row, fp4_swz),
+                           smem_desc(kb_addr + kb * 32, 16, 8 * fp4_row, fp4_swz), idesc_nvfp4(128),
+                           tmem + L::SFA_COL + 4 * kb, sfb + 4 * kb, kb > 0);
+          }
+          tc_commit(BAR(S_FULL + s));
+          tc_commit(BAR(K_EMPTY + s));
+        }
+        if (j >= 1) {
+          const int jj = j - 1, s2 = jj & 1, u2 = jj >> 1;
+          if (!mbar_wait(BAR(P_FULL + s2), u2 & 1, abort, kWaitLimitNs) ||
+              !mbar_wait(BAR(V_FULL + s2), u2 & 1, abort, kWaitLimitNs)) {
+            raise_error(abort, 2u);
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_p = tmem + L::S_COL0 + 128 * s2;
+          const uint32_t vb = sb + L::OFF_V + s2 * L::VBUF;
+          const uint32_t d_o = tmem + L::O_COL;
+          if (is_hi(jj)) {
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+              mma_bf16_ts(d_o, a_p + 8 * k, smem_desc(vb + (k >> 2) * (D * 128) + (k & 3) * 32, 16, 1024, SWZ_128B),
+                          idesc_bf16(D), (jj > 0 || k > 0) ? 1u : 0u);
+          } else {
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+              mma_e4m3_ts(d_o, a_p + 8 * k, smem_desc(vb + k * 32, 16, 1024, SWZ_128B), idesc_e4m3(D),
+                          (jj > 0 || k > 0) ? 1u : 0u);
+          }
+          tc_commit(BAR(V_EMPTY + s2));
+          tc_commit(BAR(PV_DONE));
+          if (jj == nj - 1) tc_commit(BAR(O_FINAL));
+        }
+      }
+      // every tcgen05 op issued above completes before TMEM is released
+      tc_commit(BAR(DRAIN));
+      mbar_wait(BAR(DRAIN), 0, &never, kWaitLimitNs);
+    }
+  } else {
+    // ------------------------------------------------------------ softmax
+    const int r = tid;  // query row within the tile == TMEM lane
+    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    const int row_g = i * 128 + r;
+    const float sc_hi = p.scale_log2;
+    const float sc_lo = p.scale_log2 * (p.q_gs[bhq] * p.k_gs[bhk]);
+    float m = -INFINITY, l = 0.0f;
+    bool ok = true;
+    for (int j = 0; j < nj; ++j) {
+      const int s = j & 1, u = j >> 1;
+      const bool hi = is_hi(j);
+      if (!__all_sync(0xffffffffu, mbar_wait(BAR(S_FULL + s), u & 1, abort, kWaitLimitNs))) {
+        raise_error(abort, 4u);
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t s_addr = tmem + lane_base + L::S_COL0 + 128 * s;
+      uint32_t sv[4][32];
+#pragma unroll
+      for (int c4 = 0; c4 < 4; ++c4) tmem_ld32(s_addr + 32 * c4, sv[c4]);
+      tmem_ld_wait();
+      const float sc = hi ? sc_hi : sc_lo;
+      const bool edge = (p.causal && j == i) || ((j + 1) * 128 > p.N);
+      const int lim = min(p.causal ? row_g + 1 : p.N, p.N) - j * 128;  // columns < lim are valid
+      float mx = -INFINITY;
+#pragma unroll
+      for (int c4 = 0; c4 < 4; ++c4)
+#pragma unroll
+        for (int c = 0; c < 32; ++c) {
+          float x = __uint_as_float(sv[c4][c]);
+          if (edge && (c4 * 32 + c) >= lim) x = -INFINITY;
+          sv[c4][c] = __float_as_uint(x);
+          mx = fmaxf(mx, x);
+        }
+      const float m_new = fmaxf(m, mx * sc);
+      const float alpha = (m == -INFINITY) ? 0.0f : ex2_approx(m - m_new);
+      const float nb = 8.0f - m_new;  // p * 2^8 = 2^(s * sc - m_new + 8)
+      float rs = 0.0f;
+      uint32_t pa[32], pb[32];  // packed P: e4m3 uses pa (32 columns), bf16 uses pa then pb
+      if (hi) {
+#pragma unroll
+        for (int c4 = 0; c4 < 4; ++c4)
+#pragma unroll
+          for (int c = 0; c < 32; c += 2) {
+            const float p0 = ex2_approx(fmaf(__uint_as_float(sv[c4][c]), sc, nb));
+            const float p1 = ex2_approx(fmaf(__uint_as_float(sv[c4][c + 1]), sc, nb));
+            rs += p0 + p1;
+            if (c4 < 2) pa[(c4 * 32 + c) >> 1] = cvt_bf16x2(p0, p1);
+            else pb[((c4 - 2) * 32 + c) >> 1] = cvt_bf16x2(p0, p1);
+          }
+      } else {
+#pragma unroll
+        for (int c4 = 0; c4 < 4; ++c4)
+#pragma unroll
+          for (int c = 0; c < 32; c += 4) {
+            const float p0 = ex2_approx(fmaf(__uint_as_float(sv[c4][c]), sc, nb));
+            const float p1 = ex2_approx(fmaf(__uint_as_float(sv[c4][c + 1]), sc, nb));
+            const float p2 = ex2_approx(fmaf(__uint_as_float(sv[c4][c + 2]), sc, nb));
+            const float p3 = ex2_approx(fmaf(__uint_as_float(sv[c4][c + 3]), sc, nb));
+            rs += (p0 + p1) + (p2 + p3);
+            pa[(c4 * 32 + c) >> 2] = cvt_e4m3x2(p0, p1) | (cvt_e4m3x2(p2, p3) << 16);
+          }
+      }
+      l = l * alpha + rs;
+      // rescale O when any row of this warp has a new maximum (alpha == 1 is a no-op)
+      const bool corr = (j > 0) && (alpha != 1.0f);
+      if (__any_sync(0xffffffffu, corr)) {
+        if (!__all_sync(0xffffffffu, mbar_wait(BAR(PV_DONE), (j - 1) & 1, abort, kWaitLimitNs))) {
+          raise_error(abort, 4u);
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+#pragma unroll
+        for (int c4 = 0; c4 < D / 32; ++c4) {
+          uint32_t ov[32];
+          const uint32_t o_addr = tmem + lane_base + L::O_COL + 32 * c4;
+          tmem_ld32(o_addr, ov);
+          tmem_ld_wait();
+#pragma unroll
+          for (int c = 0; c < 32; ++c) ov[c] = __float_as_uint(__uint_as_float(ov[c]) * alpha);
+          tmem_st32(o_addr, ov);
+        }
+      }
+      // P overwrites the first columns of this S buffer
+      tmem_st32(s_addr, pa);
+      if (hi) tmem_st32(s_addr + 32, pb);
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(BAR(P_FULL + s));
+      m = m_new;
+    }
+    // ---------------------------------------------------------- epilogue
+    ok = ok && __all_sync(0xffffffffu, mbar_wait(BAR(O_FINAL), 0, abort, kWaitLimitNs));
+    if (ok) {
+      tc_fence_after();
+      const float inv_l = 1.0f / l;
+      __nv_bfloat16* orow = p.o + ((size_t)bhq * p.N + row_g) * D;
+#pragma unroll
+      for (int c4 = 0; c4 < D / 32; ++c4) {
+        uint32_t ov[32];
+        tmem_ld32(tmem + lane_base + L::O_COL + 32 * c4, ov);
+        tmem_ld_wait();
+        uint32_t packed[16];
+#pragma unroll
+        for (int c = 0; c < 32; c += 2) {
+          const float a0 = __uint_as_float(ov[c]) * (vsc[c4 * 32 + c] * inv_l);
+          const float a1 = __uint_as_float(ov[c + 1]) * (vsc[c4 * 32 + c + 1] * inv_l);
+          packed[c >> 1] = cvt_bf16x2(a0, a1);
+        }
+        if (row_g < p.N) {
+          uint4* dst = reinterpret_cast<uint4*>(orow + c4 * 32);
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            dst[q] = make_uint4(packed[4 * q], packed[4 * q + 1], packed[4 * q + 2], packed[4 * q + 3]);
+        }
+      }
+      if (p.lse != nullptr && row_g < p.N)
+        p.lse[(size_t)bhq * p.N + row_g] = (m - 8.0f) * 0.69314718055994531f + logf(l);
+    } else {
+      raise_error(abort, 4u);
+    }
+  }
+
+  // ------------------------------------------------------------ teardown
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Host side: tensor maps and launch.
+// ---------------------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (fn == nullptr) {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &f, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(f);
+  }
+  return fn;
+}
+
+static bool make_map(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t d0, uint64_t d1,
+                     uint64_t d2, uint64_t s1_bytes, uint64_t s2_bytes, uint32_t b0, uint32_t b1,
+                     CUtensorMapSwizzle swz) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[3] = {d0, d1, d2};
+  cuuint64_t strides[2] = {s1_bytes, s2_bytes};
+  cuuint32_t box[3] = {b0, b1, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  return fn(m, dt, 3, const_cast<void*>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int D>
+static int launch_d(const AttnArgs& a, cudaStream_t st) {
+  using L = Layout<D>;
+  const int T = (a.N + 127) / 128, W = (T + 31) / 32;
+  const uint64_t N = (uint64_t)a.N, Np = (uint64_t)T * 128;
+  const uint64_t BHq = (uint64_t)a.B * a.Hq, BHk = (uint64_t)a.B * a.Hkv;
+  const thrift_quant& qz = *a.quant;
+  CUtensorMap m_qfp4, m_kfp4, m_qbf, m_kbf, m_vfp8, m_vbf;
+  const CUtensorMapSwizzle fp4_swz = (D == 128) ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B;
+  bool ok = true;
+  ok &= make_map(&m_qfp4, CU_TENSOR_MAP_DATA_TYPE_UINT8, qz.q_fp4, D / 2, N, BHq, D / 2, N * D / 2, D / 2, 128, fp4_swz);
+  ok &= make_map(&m_kfp4, CU_TENSOR_MAP_DATA_TYPE_UINT8, qz.k_fp4, D / 2, N, BHk, D / 2, N * D / 2, D / 2, 128, fp4_swz);
+  ok &= make_map(&m_qbf, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.q, D, N, BHq, D * 2, N * D * 2, 64, 128,
+                 CU_TENSOR_MAP_SWIZZLE_128B);
+  ok &= make_map(&m_kbf, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.k, D, N, BHk, D * 2, N * D * 2, 64, 128,
+                 CU_TENSOR_MAP_SWIZZLE_128B);
+  ok &= make_map(&m_vfp8, CU_TENSOR_MAP_DATA_TYPE_UINT8, qz.v_fp8t, Np, D, BHk, Np, Np * D, 128, D,
+                 CU_TENSOR_MAP_SWIZZLE_128B);
+  ok &= make_map(&m_vbf, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, qz.v_st, Np, D, BHk, Np * 2, Np * D * 2, 64, D,
+                 CU_TENSOR_MAP_SWIZZLE_128B);
+  if (!ok) return THRIFT_ERR_CUDA;
+  Params p;
+  p.q_sf_mma = qz.q_sf_mma;
+  p.k_sf_mma = qz.k_sf_mma;
+  p.q_gs = qz.q_gs;
+  p.k_gs = qz.k_gs;
+  p.v_exp = qz.v_exp;
+  p.mask = a.mask;
+  p.o = reinterpret_cast<__nv_bfloat16*>(a.o);
+  p.lse = a.lse;
+  p.B = a.B; p.Hq = a.Hq; p.Hkv = a.Hkv; p.N = a.N; p.T = T; p.W = W; p.causal = a.causal;
+  const float scale = a.softmax_scale > 0.0f ? a.softmax_scale : 1.0f / sqrtf((float)D);
+  p.scale_log2 = scale * 1.4426950408889634f;
+  if (cudaFuncSetAttribute(attn_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::DYN) != cudaSuccess)
+    return THRIFT_ERR_CUDA;
+  const unsigned grid = (unsigned)(BHq * (uint64_t)T);
+  attn_fwd_kernel<D><<<grid, kThreads, L::DYN, st>>>(m_qfp4, m_kfp4, m_qbf, m_kbf, m_vfp8, m_vbf, p);
+  count_launches(1);
+  return cudaGetLastError() == cudaSuccess ? THRIFT_OK : THRIFT_ERR_CUDA;
+}
+
+}  // namespace attn
+
+int launch_attn(const AttnArgs& a, cudaStream_t s) {
+  if (a.d == 128) return attn::launch_d<128>(a, s);
+  return attn::launch_d<64>(a, s);
+}
+
+cudaError_t read_and_clear_device_error(cudaStream_t s, uint32_t* word) {
+  cudaError_t e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return e;
+  uint32_t w = 0;
+  e = cudaMemcpyFromSymbol(&w, g_attn_error_word, sizeof(w));
+  if (e != cudaSuccess) return e;
+  if (w != 0) {
+    const uint32_t zero = 0;
+    e = cudaMemcpyToSymbol(g_attn_error_word, &zero, sizeof(zero));
+  }
+  *word = w;
+  return e;
+}
+
+}  // namespace thrift

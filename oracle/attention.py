@@ -40,7 +40,7 @@ import numpy as np
 import torch
 
 from .formats import bf16_round, e4m3_decode, e4m3_encode
-from .quantize import nvfp4_dequantize
+from .quantize import fp8_v_quantize, nvfp4_dequantize, nvfp4_quantize, tensor_scale
 from .select import mask_bit
 
 
@@ -51,7 +51,13 @@ def _f64(x) -> np.ndarray:
 
 
 class Operands:
-    """The FP64 views of one problem that the tile loop reads, built per head on demand."""
+    """The FP64 views of one problem that the tile loop reads, built per head on demand.
+
+    ``quant`` may hold the full quantised operands (as ``oracle.quantize.quantize``
+    returns them); when it is None each head is quantised when first needed,
+    with the same per-head arithmetic (query tiles use the head's tensor scale
+    from the whole head and quantise only their own rows).
+    """
 
     def __init__(self, q, k, v, quant, causal: bool, sm_scale: float = 0.0):
         self._q, self._k, self._v = q, k, v
@@ -65,26 +71,41 @@ class Operands:
         self._qc = {}
         self._kc = {}
 
-    def q_views(self, b: int, h: int):
-        key = (b, h)
-        if key not in self._qc:
-            qz = self.quant
-            q_hi = _f64(self._q[b, h])
-            q_lo = nvfp4_dequantize(qz["q_codes"][b:b + 1, h:h + 1], qz["q_sf"][b:b + 1, h:h + 1],
+    def q_tile(self, b: int, h: int, r0: int, r1: int):
+        qz = self.quant
+        q_hi = _f64(self._q[b, h, r0:r1])
+        if qz is not None:
+            q_lo = nvfp4_dequantize(qz["q_codes"][b:b + 1, h:h + 1, r0:r1], qz["q_sf"][b:b + 1, h:h + 1, r0:r1],
                                     np.asarray(qz["q_g"])[b:b + 1, h:h + 1])[0, 0]
-            self._qc = {key: (q_hi, q_lo)}
-        return self._qc[key]
+        else:
+            key = (b, h)
+            if key not in self._qc:
+                head = self._q[b, h]
+                amax = float(head.abs().max()) if isinstance(head, torch.Tensor) else float(np.abs(head).max())
+                self._qc = {key: tensor_scale(np.array([[amax]], dtype=np.float32))}
+            g = self._qc[key]
+            rows = self._q[b:b + 1, h:h + 1, r0:r1]
+            codes, sf, g = nvfp4_quantize(rows, g=g)
+            q_lo = nvfp4_dequantize(codes, sf, g)[0, 0]
+        return q_hi, q_lo
 
     def kv_views(self, b: int, hk: int):
         key = (b, hk)
         if key not in self._kc:
             qz = self.quant
+            if qz is None:
+                codes, sf, g = nvfp4_quantize(self._k[b:b + 1, hk:hk + 1])
+                v_code, v_exp, _ = fp8_v_quantize(self._v[b:b + 1, hk:hk + 1])
+                qz = dict(k_codes=codes, k_sf=sf, k_g=g, v_code=v_code, v_exp=v_exp)
+                bb, hh = 0, 0
+            else:
+                bb, hh = b, hk
             k_hi = _f64(self._k[b, hk])
-            k_lo = nvfp4_dequantize(qz["k_codes"][b:b + 1, hk:hk + 1], qz["k_sf"][b:b + 1, hk:hk + 1],
-                                    np.asarray(qz["k_g"])[b:b + 1, hk:hk + 1])[0, 0]
+            k_lo = nvfp4_dequantize(qz["k_codes"][bb:bb + 1, hh:hh + 1], qz["k_sf"][bb:bb + 1, hh:hh + 1],
+                                    np.asarray(qz["k_g"])[bb:bb + 1, hh:hh + 1])[0, 0]
             v_hi = _f64(self._v[b, hk])
-            e = np.asarray(qz["v_exp"], dtype=np.int64)[b, hk]
-            v_lo = e4m3_decode(qz["v_code"][b, hk]) * np.ldexp(1.0, e)[None, :]
+            e = np.asarray(qz["v_exp"], dtype=np.int64)[bb, hh]
+            v_lo = e4m3_decode(qz["v_code"][bb, hh]) * np.ldexp(1.0, e)[None, :]
             self._kc = {key: (k_hi, k_lo, v_hi, v_lo)}
         return self._kc[key]
 
@@ -97,10 +118,8 @@ def attn_query_tile(ops: Operands, mask, b: int, h: int, i: int,
     r1 = min(ops.N, r0 + 128)
     rows = np.arange(r0, r1)
     nr = r1 - r0
-    q_hi_all, q_lo_all = ops.q_views(b, h)
+    q_hi, q_lo = ops.q_tile(b, h, r0, r1)
     k_hi, k_lo, v_hi, v_lo = ops.kv_views(b, hk)
-    q_hi = q_hi_all[r0:r1]
-    q_lo = q_lo_all[r0:r1]
     m = np.full(nr, -np.inf)
     l = np.zeros(nr)
     O = np.zeros((nr, ops.d))
@@ -140,6 +159,8 @@ def attn_query_tile(ops: Operands, mask, b: int, h: int, i: int,
 def attn_forward(q, k, v, quant, mask, causal: bool, sm_scale: float = 0.0,
                  sigma: int = 8, p_cast: bool = True, tiles=None):
     """Full (or sampled) mixed-precision attention forward.
+
+    ``quant``: the quantised operands, or None to quantise each head on demand.
 
     ``tiles``: optional list of (b, h, i) query tiles; when given only those
     rows of the output are filled (the rest stay NaN).

@@ -43,17 +43,27 @@ def _as_f32(x) -> np.ndarray:
     return np.asarray(x, dtype=np.float32)
 
 
-def nvfp4_quantize(x):
+def tensor_scale(amax) -> np.ndarray:
+    """Per-head tensor scale g = amax / 2688 in FP32 (1 for an all-zero head)."""
+    amax = np.asarray(amax, dtype=F32)
+    return np.where(amax > 0, (amax / F32(2688.0)).astype(F32), F32(1.0)).astype(F32)
+
+
+def nvfp4_quantize(x, g=None):
     """NVFP4-quantise ``x[B,H,N,d]`` (BF16 values) per (B,H) head.
 
+    ``g`` (optional, [B,H]) supplies the head's tensor scale when ``x`` holds
+    only some rows of the head; by default it comes from ``x`` itself.
     Returns (codes[B,H,N,d] uint8 0..15, sf[B,H,N,d/16] uint8 e4m3 codes,
     g[B,H] float32).
     """
     x = _as_f32(x)
     B, H, N, d = x.shape
     assert d % 16 == 0
-    amax = np.abs(x).reshape(B, H, -1).max(axis=2) if N > 0 else np.zeros((B, H), F32)
-    g = np.where(amax > 0, (amax / F32(2688.0)).astype(F32), F32(1.0)).astype(F32)
+    if g is None:
+        amax = np.abs(x).reshape(B, H, -1).max(axis=2) if N > 0 else np.zeros((B, H), F32)
+        g = tensor_scale(amax)
+    g = np.asarray(g, dtype=F32)
     blk = x.reshape(B, H, N, d // 16, 16)
     amax_b = np.abs(blk).max(axis=4)                                 # f32, exact
     six_g = (F32(6.0) * g).astype(F32)                               # f32 product

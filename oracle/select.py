@@ -85,39 +85,53 @@ def budget_for_row(n_i: int, n_forced: int, budget_bp: int, budget_tiles: int) -
     return min(n_i, max(n_forced, want))
 
 
-def select_rows(scores, causal: bool, budget_bp: int, budget_tiles: int):
-    """scores[B,Hq,T,T] -> (mask[B,Hq,T,W] uint32, counts[B,Hq,T] int32)."""
+def select_rows(scores, causal: bool, budget_bp: int, budget_tiles: int, rows=None):
+    """scores[B,Hq,T,T] -> (mask[B,Hq,T,W] uint32, counts[B,Hq,T] int32).
+
+    ``rows``: optional list of (b, h, i) query tiles to fill (others stay 0).
+    """
     scores = np.asarray(scores, dtype=F32)
     B, H, T, _ = scores.shape
     W = (T + 31) // 32
     mask = np.zeros((B, H, T, W), dtype=np.uint32)
     counts = np.zeros((B, H, T), dtype=np.int32)
-    for b in range(B):
-        for h in range(H):
-            for i in range(T):
-                n_i = i + 1 if causal else T
-                forced = sorted({0, i} & set(range(n_i)))
-                k_i = budget_for_row(n_i, len(forced), budget_bp, budget_tiles)
-                chosen = []
-                if k_i > 0:
-                    chosen = list(forced)
-                    rest = [j for j in range(n_i) if j not in forced]
-                    s = scores[b, h, i, rest].astype(np.float64)   # -0 == +0 in comparisons
-                    order = np.lexsort((np.asarray(rest), -s))     # score desc, then index asc
-                    chosen += [rest[o] for o in order[: k_i - len(forced)]]
-                for j in chosen:
-                    mask[b, h, i, j // 32] |= np.uint32(1) << np.uint32(j % 32)
-                counts[b, h, i] = len(chosen)
+    if rows is None:
+        rows = [(b, h, i) for b in range(B) for h in range(H) for i in range(T)]
+    for (b, h, i) in rows:
+        n_i = i + 1 if causal else T
+        forced = sorted({0, i} & set(range(n_i)))
+        k_i = budget_for_row(n_i, len(forced), budget_bp, budget_tiles)
+        chosen = []
+        if k_i > 0:
+            chosen = list(forced)
+            rest = [j for j in range(n_i) if j not in forced]
+            s = scores[b, h, i, rest].astype(np.float64)   # -0 == +0 in comparisons
+            order = np.lexsort((np.asarray(rest), -s))     # score desc, then index asc
+            chosen += [rest[o] for o in order[: k_i - len(forced)]]
+        for j in chosen:
+            mask[b, h, i, j // 32] |= np.uint32(1) << np.uint32(j % 32)
+        counts[b, h, i] = len(chosen)
     return mask, counts
 
 
-def select(q, k, causal: bool, budget_bp: int, budget_tiles: int = 0):
-    """The library's ``thrift_select``: pooled scores -> BF16 tile mask."""
+def select(q, k, causal: bool, budget_bp: int, budget_tiles: int = 0, rows=None):
+    """The library's ``thrift_select``: pooled scores -> BF16 tile mask.
+
+    ``rows``: optional list of (b, h, i) query tiles to compute (others stay 0).
+    """
     qp = pool_tiles(q)
     kp = pool_tiles(k)
     Hq, Hkv = qp.shape[1], kp.shape[1]
-    sc = tile_scores(qp, kp, Hq, Hkv)
-    mask, counts = select_rows(sc, causal, budget_bp, budget_tiles)
+    if rows is None:
+        sc = tile_scores(qp, kp, Hq, Hkv)
+    else:
+        # scores only for the requested query tiles (same products and order)
+        B, _, T, d = qp.shape
+        sc = np.zeros((B, Hq, T, T), dtype=F32)
+        G = Hq // Hkv
+        for (b, h, i) in rows:
+            sc[b, h, i] = tile_scores(qp[b:b + 1, h:h + 1, i:i + 1], kp[b:b + 1, h // G:h // G + 1], 1, 1)[0, 0, 0]
+    mask, counts = select_rows(sc, causal, budget_bp, budget_tiles, rows)
     return dict(qp=qp, kp=kp, scores=sc, mask=mask, counts=counts)
 
 

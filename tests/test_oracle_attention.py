@@ -147,3 +147,13 @@ def test_sampled_tiles_match_full_run():
     assert np.array_equal(Os[0, 1, 256:384], O[0, 1, 256:384])
     assert np.array_equal(Os[0, 3, 0:128], O[0, 3, 0:128])
     assert np.isnan(Os[0, 0]).all()
+
+
+def test_on_demand_quantisation_matches_full_quantisation():
+    q, k, v = _problem(N=400, seed=8)
+    qz = quantize(q, k, v)
+    sel = select(q, k, True, budget_bp=1500)
+    tiles = [(0, 0, 3), (0, 2, 1), (0, 3, 2)]
+    O1, l1 = attn_forward(q, k, v, qz, sel["mask"], True, tiles=tiles)
+    O2, l2 = attn_forward(q, k, v, None, sel["mask"], True, tiles=tiles)
+    assert np.array_equal(np.nan_to_num(O1, nan=7.0), np.nan_to_num(O2, nan=7.0))

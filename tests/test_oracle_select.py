@@ -171,3 +171,13 @@ def test_pooled_means_close_to_float64(rng):
     for t in range(3):
         want = xf[:, :, t * 128:min(300, (t + 1) * 128)].mean(axis=2)
         assert np.allclose(p[:, :, t], want, rtol=1e-5, atol=1e-6)
+
+
+def test_row_subset_matches_full_selection():
+    q, k = _random_problem(seed=11, N=1200)
+    full = select(q, k, True, 1500)
+    rows = [(0, 0, 3), (0, 3, 9), (0, 1, 0)]
+    part = select(q, k, True, 1500, rows=rows)
+    for (b, h, i) in rows:
+        assert np.array_equal(part["mask"][b, h, i], full["mask"][b, h, i])
+        assert part["counts"][b, h, i] == full["counts"][b, h, i]
