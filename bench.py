@@ -1,0 +1,432 @@
+"""Benchmark: mixed FP4/BF16 attention forward (prefill) on B200.
+
+One step = the whole hot path on one batch of synthetic input resident in
+HBM: thrift_quantize -> thrift_select -> thrift_attn_fwd.  Default workload:
+causal GQA prefill, B=1, Hq=32, Hkv=8, N=32768, d=128, 5% BF16 tile budget.
+
+Metric: effective attention TFLOP/s, causal-adjusted (2*B*Hq*N^2*d FLOPs per
+step for causal runs, 4*B*Hq*N^2*d otherwise) over the device-timed step.
+
+Multi-GPU (torchrun, one process per GPU): every rank runs its own full
+problem (heads and batches are independent; no collective on the data
+path), so scaling is weak and value = all ranks' FLOPs / max-over-ranks time.
+
+`--impl reference` times the CPU oracle (the statement of the method the
+library is checked against) on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+from mixed_precision_bit_quant_b200 import workloads  # noqa: E402
+
+METRIC = "attn TFLOPS (causal-adj) & % of mixed FP4/BF16 roofline, N=32K, 5% BF16"
+UNIT = "TFLOP/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def _dist():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def hi_lo_pairs(w: workloads.Workload):
+    """(BF16 pairs, FP4 pairs) the budget rule yields for workload w (closed form)."""
+    T = w.T
+    hi = lo = 0
+    for i in range(T):
+        n_i = i + 1 if w.causal else T
+        nf = 1 if i == 0 else 2
+        if w.budget_tiles > 0:
+            k = min(n_i, max(nf, w.budget_tiles))
+        elif w.budget_bp <= 0:
+            k = 0
+        elif w.budget_bp >= 10000:
+            k = n_i
+        else:
+            k = min(n_i, max(nf, (w.budget_bp * n_i + 9999) // 10000))
+        hi += k
+        lo += n_i - k
+    return hi * w.B * w.Hq, lo * w.B * w.Hq
+
+
+def attn_roofline(w: workloads.Workload, peaks: dict, key: str = "bf16_tflops"):
+    """Mixed tensor roofline of the attention kernel.
+
+    Per computed 128x128 tile pair: F = 2*128*128*d FLOPs for Q K^T and the
+    same for P V.  FP4 pairs run Q K^T at the FP4 rate and P V at the FP8
+    rate; BF16 pairs run both at the BF16 rate.  Rates: the measured BF16
+    GEMM peak, times 2 (FP8) and 4 (FP4), the nominal dense ratios.
+    """
+    hi, lo = hi_lo_pairs(w)
+    F = 2.0 * 128 * 128 * w.d
+    p16 = peaks[key] * 1e12
+    p8, p4 = 2 * p16, 4 * p16
+    t = lo * (F / p4 + F / p8) + hi * (2 * F / p16)
+    flops = (hi + lo) * 2 * F
+    return dict(flops=flops, t_roof=t, peak=flops / t, hi=hi, lo=lo)
+
+
+def attn_algorithmic_bytes(w: workloads.Workload, hi: int, lo: int) -> float:
+    """Compulsory HBM bytes of one attention launch (each operand read once, O written once)."""
+    B, Hq, Hkv, N, d = w.B, w.Hq, w.Hkv, w.N, w.d
+    q = B * Hq * N * d * (2 + 0.5 + 1 / 16)
+    kv = B * Hkv * N * d * (2 + 0.5 + 1 / 16 + 1 + 2)
+    o = B * Hq * N * d * 2
+    return q + kv + o
+
+
+def quantize_algorithmic_bytes(w):
+    B, Hq, Hkv, N, d = w.B, w.Hq, w.Hkv, w.N, w.d
+    Np = w.T * 128
+    inp = (B * Hq + 2 * B * Hkv) * N * d * 2
+    out = (B * Hq + B * Hkv) * (N * d / 2 + N * d / 16 + w.T * 128 * d / 16) + B * Hkv * d * Np * 3
+    return inp + out
+
+
+def select_algorithmic_bytes(w):
+    return (w.B * w.Hq + w.B * w.Hkv) * w.N * w.d * 2
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled every 100 ms in a background process."""
+
+    FIELDS = ("index,timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+        self.t_start = self.t_stop = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+            return
+        self._th = threading.Thread(target=self._read, daemon=True)
+        self._th.start()
+
+    def _read(self):
+        for ln in self.proc.stdout:
+            self.lines.append((time.time(), ln.strip()))
+
+    def mark_start(self):
+        self.t_start = time.time()
+
+    def mark_stop(self):
+        self.t_stop = time.time()
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        if not self.lines:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        inwin = [(t, l) for (t, l) in self.lines if self.t_start - 0.05 <= t <= self.t_stop + 0.15]
+        if not inwin:
+            # nearest sample to the window's middle
+            mid = 0.5 * (self.t_start + self.t_stop)
+            inwin = [min(self.lines, key=lambda x: abs(x[0] - mid))]
+        sms, maxs, power, reasons = [], [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for _, l in inwin:
+            f = [x.strip() for x in l.split(",")]
+            try:
+                sms.append(float(f[2]))
+                maxs.append(float(f[3]))
+                power.append(float(f[4]))
+            except (ValueError, IndexError):
+                continue
+            for n, v in zip(names, f[6:10]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sms) if sms else None, "sm_max_mhz": max(maxs) if maxs else None,
+                "power_w_max": max(power) if power else None, "reasons": sorted(reasons), "samples": len(sms)}
+
+
+def oracle_sample_run(w: workloads.Workload, q, k, v, tiles):
+    """Time the CPU oracle on `tiles`: for each (b, h, i), the single-head problem
+    (q head h, its kv head) runs select + mixed attention with on-demand
+    quantisation.  Heads are independent, so this is the same arithmetic as
+    the full problem restricted to those rows.  Single-threaded BLAS."""
+    from threadpoolctl import threadpool_limits
+
+    from oracle import attention as oatt
+    from oracle import select as osel
+    G = w.Hq // w.Hkv
+    t0 = time.perf_counter()
+    with threadpool_limits(limits=1):
+        for (b, h, i) in tiles:
+            qs = q[b:b + 1, h:h + 1]
+            ks = k[b:b + 1, h // G:h // G + 1]
+            vs = v[b:b + 1, h // G:h // G + 1]
+            sel = osel.select(qs, ks, w.causal, w.budget_bp, w.budget_tiles, rows=[(0, 0, i)])
+            oatt.attn_forward(qs, ks, vs, None, sel["mask"], w.causal, tiles=[(0, 0, i)])
+    dt = time.perf_counter() - t0
+    flops = 0.0
+    for (_, _, i) in tiles:
+        r0, r1 = i * 128, min(w.N, (i + 1) * 128)
+        for r in range(r0, r1):
+            flops += 4.0 * w.d * ((r + 1) if w.causal else w.N)
+    return dt, flops
+
+
+def cpu_baseline(w, q, k, v, n_tiles: int, seed: int = 1):
+    tiles = workloads.sample_query_tiles(w, n_tiles, seed=seed)
+    dt, flops = oracle_sample_run(w, q, k, v, tiles)
+    return {"value": flops / dt / 1e12, "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": f"{len(tiles)} query tiles (seed {seed}) of {w.name}, each as its single-head problem: "
+                      f"pool/score/select + quantise the head + mixed attention of the tile; "
+                      f"{dt:.1f} s, single-threaded numpy (FP32 decisions, FP64 attention)",
+            "seconds": dt}
+
+
+def run_reference(args, w):
+    rank, world, _ = _dist()
+    if rank != 0:
+        return 0
+    q, k, v = workloads.generate(w)
+    vals = []
+    cb = None
+    n_tiles = args.ref_tiles
+    for s in range(args.warmup + args.steps):
+        tiles = workloads.sample_query_tiles(w, n_tiles, seed=1 + s)
+        dt, flops = oracle_sample_run(w, q, k, v, tiles)
+        if s >= args.warmup:
+            vals.append((dt, flops))
+    tot_t = sum(d for d, _ in vals)
+    tot_f = sum(f for _, f in vals)
+    value = tot_f / tot_t / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot_t / max(1, len(vals)),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": config_of(w, world),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
+                         "sample": f"{n_tiles} query tiles per step (seeds 1..), select + mixed attention"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def config_of(w, world):
+    return {"workload": f"{w.name}: causal={int(w.causal)} B={w.B} Hq={w.Hq} Hkv={w.Hkv} N={w.N} d={w.d} "
+                        f"budget_bp={w.budget_bp} budget_tiles={w.budget_tiles}",
+            "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.N, "d": w.d, "causal": w.causal,
+            "budget_bp": w.budget_bp, "parallelism": f"independent problem per rank x{world}",
+            "l2": "inputs larger than L2 (Q alone is 268 MB at N=32K); no flush between steps"}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="thrift", choices=["thrift", "reference"])
+    ap.add_argument("--workload", default="llm32k", choices=sorted(workloads.WORKLOADS))
+    ap.add_argument("--budget-bp", type=int, default=None)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-clocks", action="store_true")
+    ap.add_argument("--cpu-tiles", type=int, default=16)
+    ap.add_argument("--ref-tiles", type=int, default=1)
+    args = ap.parse_args()
+    w = workloads.WORKLOADS[args.workload]
+    if args.budget_bp is not None:
+        w = w.with_budget(bp=args.budget_bp)
+    if args.impl == "reference":
+        return run_reference(args, w)
+
+    import mixed_precision_bit_quant_b200 as mq
+
+    rank, world, local = _dist()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    pg = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+        pg = dist
+    peaks, peak_src = _peaks()
+
+    q_h, k_h, v_h = workloads.generate(w)
+    q, k, v = (t.to(dev) for t in (q_h, k_h, v_h))
+    quant = mq.alloc_quantized(mq.shape_of(q, k, w.causal), dev)
+    shape = mq.shape_of(q, k, w.causal)
+    ws_q = torch.empty(max(16, mq.workspace_bytes(shape, mq.OP_QUANTIZE)), dtype=torch.uint8, device=dev)
+    ws_s = torch.empty(max(16, mq.workspace_bytes(shape, mq.OP_SELECT)), dtype=torch.uint8, device=dev)
+    T, W = w.T, (w.T + 31) // 32
+    mask = torch.empty((w.B, w.Hq, T, W), dtype=torch.int32, device=dev)
+    counts = torch.empty((w.B, w.Hq, T), dtype=torch.int32, device=dev)
+    o = torch.empty_like(q)
+    stream = torch.cuda.current_stream(dev)
+
+    ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+    K = args.steps
+    marks = [(ev(), ev(), ev(), ev()) for _ in range(K)]
+
+    def step(m=None):
+        if m is not None:
+            m[0].record(stream)
+        mq.quantize(q, k, v, w.causal, out=quant, ws=ws_q)
+        if m is not None:
+            m[1].record(stream)
+        mq.select(q, k, w.causal, w.budget_bp, w.budget_tiles, mask=mask, counts=counts, ws=ws_s)
+        if m is not None:
+            m[2].record(stream)
+        mq.attn_fwd(q, k, quant, mask, w.causal, o=o)
+        if m is not None:
+            m[3].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    status, word = mq.device_status()
+    if status != 0:
+        raise RuntimeError(f"device watchdog raised {word:#x} during warm-up")
+
+    sampler = None if args.no_clocks else ClockSampler(local)
+    if sampler:
+        sampler.start()
+        time.sleep(0.6)  # nvidia-smi start-up
+    if pg:
+        pg.barrier()
+    torch.cuda.synchronize(dev)
+    n0 = mq.launch_count()
+    t_begin, t_end = ev(), ev()
+    if sampler:
+        sampler.mark_start()
+    t_begin.record(stream)
+    for s in range(K):
+        step(marks[s])
+    t_end.record(stream)
+    torch.cuda.synchronize(dev)
+    if sampler:
+        sampler.mark_stop()
+    if pg:
+        pg.barrier()
+    launches = mq.launch_count() - n0
+    status, word = mq.device_status()
+    if status != 0:
+        raise RuntimeError(f"device watchdog raised {word:#x} in the timed region")
+    if sampler:
+        time.sleep(0.2)
+        sampler.stop()
+    total_ms = t_begin.elapsed_time(t_end)
+    if pg:
+        tt = torch.tensor([total_ms], device=dev)
+        pg.all_reduce(tt, op=pg.ReduceOp.MAX)
+        total_ms = float(tt.item())
+    ms_step = total_ms / K
+    q_ms = statistics.mean(m[0].elapsed_time(m[1]) for m in marks)
+    s_ms = statistics.mean(m[1].elapsed_time(m[2]) for m in marks)
+    a_ms = statistics.mean(m[2].elapsed_time(m[3]) for m in marks)
+
+    eff_flops = w.causal_adjusted_flops()
+    value = world * eff_flops / (ms_step * 1e-3) / 1e12
+    roof = attn_roofline(w, peaks, "bf16_tflops")
+    achieved = roof["flops"] / (a_ms * 1e-3) / 1e12
+    peak = roof["peak"] / 1e12
+
+    # ------------------------------------------------ end to end through host buffers
+    e2e = None
+    if not args.no_e2e:
+        qp, kp, vp = (t.pin_memory() for t in (q_h, k_h, v_h))
+        o_host = torch.empty(q_h.shape, dtype=torch.bfloat16).pin_memory()
+        ke = max(3, min(10, K))
+        for it in range(2 + ke):
+            if it == 2:
+                torch.cuda.synchronize(dev)
+                if pg:
+                    pg.barrier()
+                e0, e1 = ev(), ev()
+                e0.record(stream)
+            q.copy_(qp, non_blocking=True)
+            k.copy_(kp, non_blocking=True)
+            v.copy_(vp, non_blocking=True)
+            step()
+            o_host.copy_(o, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        e_ms = e0.elapsed_time(e1) / ke
+        if pg:
+            tt = torch.tensor([e_ms], device=dev)
+            pg.all_reduce(tt, op=pg.ReduceOp.MAX)
+            e_ms = float(tt.item())
+        h2d = sum(t.numel() * t.element_size() for t in (q_h, k_h, v_h))
+        e2e = {"value": world * eff_flops / (e_ms * 1e-3) / 1e12, "unit": UNIT, "ms_per_step": e_ms,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": o_host.numel() * 2,
+               "api": "mixed_precision_bit_quant_b200.quantize/select/attn_fwd (C ABI) with pinned host copies"}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(w, q_h, k_h, v_h, args.cpu_tiles)
+
+    if rank == 0:
+        hbm = peaks["hbm_gbs"]
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
+            "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "nvfp4/e4m3/bf16 (fp32 accumulate)", "data": "synthetic", "config": config_of(w, world),
+            "roofline": {"bound": "tensor", "kernel": "attn_fwd_kernel<128>", "achieved": achieved, "peak": peak,
+                         "unit": "TFLOP/s", "frac": achieved / peak, "traffic": None,
+                         "peak_source": f"{peak_src} bf16 {peaks['bf16_tflops']} TF/s burst; FP8 = 2x, FP4 = 4x "
+                                        f"(nominal dense ratios); BF16 pairs {roof['hi']}, FP4 pairs {roof['lo']}",
+                         "t_roof_ms": roof["t_roof"] * 1e3, "algorithmic_flops": roof["flops"]},
+            "stages_ms": {"quantize": q_ms, "select": s_ms, "attn_fwd": a_ms},
+            "stages_gbs": {"quantize": quantize_algorithmic_bytes(w) / (q_ms * 1e-3) / 1e9,
+                           "select": select_algorithmic_bytes(w) / (s_ms * 1e-3) / 1e9,
+                           "hbm_peak": hbm},
+            "attn_only_tflops_causal_adj": eff_flops / (a_ms * 1e-3) / 1e12,
+            "attn_algorithmic_bytes": attn_algorithmic_bytes(w, roof["hi"], roof["lo"]),
+            "gpu_launches": launches,
+            "clocks": sampler.summary() if sampler else None,
+            "e2e": e2e,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    if pg:
+        pg.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())
