@@ -120,6 +120,31 @@ THRIFT_API thrift_status thrift_quantize(const thrift_shape *shape, const void *
                               size_t ws_bytes, void *stream);
 
 /*
+ * thrift_quantize without a workspace argument.  The pages have no
+ * counterpart of this call; it exists for callers that cannot allocate device
+ * memory, e.g. a C host program that owns only its input and output buffers,
+ * code running in a host callback or allocator hook where allocating is not
+ * allowed, or a process whose device memory pool belongs to another component.
+ *
+ * Results are identical to thrift_quantize.  The per-head and per-channel amax
+ * accumulators live in a fixed array inside the library: 65536 32-bit words
+ * (256 KB) of device memory on every GPU that loads the library, held until the
+ * process exits.  A shape needing more than that, i.e. with
+ * B*Hq + B*Hkv + B*Hkv*d > 65536, is rejected with THRIFT_ERR_UNSUPPORTED.
+ * Nothing is allocated or freed by this call.
+ *
+ * The first call on a device looks up the array's device address with that
+ * device current (a one-time set-up per device); make that first call before
+ * any stream capture.  All calls share the array and each clears the words it
+ * uses before it uses them, so calls whose work can overlap on the GPU (other
+ * streams, other host threads on the same device) race on it and must be
+ * serialised by the caller.
+ */
+THRIFT_API thrift_status thrift_quantize_noalloc(const thrift_shape *shape, const void *q,
+                                                const void *k, const void *v,
+                                                const thrift_quant *out, void *stream);
+
+/*
  * Stage 1: the BF16 tile-pair bitmask.
  * For every (b, hq, query tile i): pooled means qp_i, kp_j (FP32 column sums
  * over the tile's valid rows in ascending order, divided by the row count);

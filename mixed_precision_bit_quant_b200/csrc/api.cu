@@ -97,6 +97,24 @@ thrift_status thrift_quantize(const thrift_shape* shape, const void* q, const vo
   return launch_quantize(a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? THRIFT_OK : THRIFT_ERR_CUDA;
 }
 
+thrift_status thrift_quantize_noalloc(const thrift_shape* shape, const void* q, const void* k, const void* v,
+                                      const thrift_quant* out, void* stream) {
+  int e = check_shape(shape);
+  if (e) return (thrift_status)e;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v)) return THRIFT_ERR_INVALID;
+  if ((e = check_quant(out))) return (thrift_status)e;
+  const size_t words = thrift_workspace_bytes(shape, THRIFT_OP_QUANTIZE) / sizeof(uint32_t);
+  if (words > noalloc_scratch_words()) return THRIFT_ERR_UNSUPPORTED;
+  QuantArgs a;
+  a.B = shape->B; a.Hq = shape->Hq; a.Hkv = shape->Hkv; a.N = shape->N; a.d = shape->d;
+  a.q = static_cast<const __nv_bfloat16*>(q);
+  a.k = static_cast<const __nv_bfloat16*>(k);
+  a.v = static_cast<const __nv_bfloat16*>(v);
+  a.out = *out;
+  a.amax_ws = nullptr;
+  return launch_quantize_noalloc(a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? THRIFT_OK : THRIFT_ERR_CUDA;
+}
+
 thrift_status thrift_select(const thrift_shape* shape, const void* q, const void* k, int32_t budget_bp,
                             int32_t budget_tiles, uint32_t* mask, int32_t* counts, void* ws, size_t ws_bytes,
                             void* stream) {

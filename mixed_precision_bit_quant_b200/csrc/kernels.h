@@ -17,6 +17,9 @@ struct QuantArgs {
   uint32_t* amax_ws;  // [B*Hq + B*Hkv + B*Hkv*d]
 };
 cudaError_t launch_quantize(const QuantArgs& a, cudaStream_t s);
+// Same as launch_quantize, with the amax scratch in the library's static device array.
+cudaError_t launch_quantize_noalloc(QuantArgs a, cudaStream_t s);
+size_t noalloc_scratch_words();
 
 struct SelectArgs {
   int B, Hq, Hkv, N, d, causal;

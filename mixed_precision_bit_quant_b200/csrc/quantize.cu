@@ -8,6 +8,8 @@
 //
 // All kernels are HBM-bound: 16-byte loads, warp-level max reductions, one
 // atomic per warp for the amax passes.
+#include <mutex>
+
 #include "dev.cuh"
 #include "kernels.h"
 
@@ -246,6 +248,54 @@ cudaError_t launch_quantize(const QuantArgs& a, cudaStream_t s) {
     count_launches(3);
   }
   return cudaGetLastError();
+}
+
+
+// ---------------------------------------------------------------------------
+// Workspace-free quantisation.  Some callers cannot hand the library a device
+// workspace: code that runs where device allocation is not allowed or not
+// possible (for example inside a host callback or a custom allocator hook, in
+// a process whose memory pool is owned by someone else, or in a C host program
+// that only holds the input and output buffers).  For them the amax
+// accumulators live in a fixed array in this library's device memory.
+//
+// The array holds kNoAllocWords 32-bit words (256 KB) on every GPU that loads
+// the library, for the life of the process.  All calls share it: each call
+// clears the words it uses before use, and calls whose work overlaps on the
+// GPU (different streams, or different host threads on one device) race on it.
+// ---------------------------------------------------------------------------
+constexpr size_t kNoAllocWords = 65536;
+static __device__ __align__(256) uint32_t g_noalloc_amax[kNoAllocWords];
+
+namespace {
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+uint32_t* g_noalloc_ptr[kMaxDevices] = {};
+}  // namespace
+
+size_t noalloc_scratch_words() { return kNoAllocWords; }
+
+// Host code must not pass `g_noalloc_amax` itself to a kernel: on the host that
+// name is only a stand-in for the device array.  The device address is looked
+// up once per device, with that device current, on the first call made on it.
+cudaError_t launch_quantize_noalloc(QuantArgs a, cudaStream_t s) {
+  int dev = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return err;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  uint32_t* ptr = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (g_noalloc_ptr[dev] == nullptr) {
+      void* p = nullptr;
+      err = cudaGetSymbolAddress(&p, g_noalloc_amax);
+      if (err != cudaSuccess) return err;
+      g_noalloc_ptr[dev] = static_cast<uint32_t*>(p);
+    }
+    ptr = g_noalloc_ptr[dev];
+  }
+  a.amax_ws = ptr;  // launch_quantize clears the words it uses before the amax passes
+  return launch_quantize(a, s);
 }
 
 }  // namespace thrift
