@@ -23,6 +23,7 @@
 // TMEM columns: S double buffer [0,256), O [256, 256+D), scale factors after.
 // The S computation of tile j+1 overlaps the softmax of tile j.
 #include <cuda.h>
+#include <stdlib.h>
 
 #include "dev.cuh"
 #include "kernels.h"
@@ -34,8 +35,9 @@ __device__ uint32_t g_attn_error_word;
 namespace attn {
 
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s per wait: far above any legitimate wait
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;  // 8 softmax warps, 1 TMA warp, 1 MMA warp
 constexpr int kMaxW = 128;                          // mask words per query tile (T <= 4096)
+constexpr int kDefaultPolyPairs = 0;
 
 enum Bar : int {
   Q_FULL = 0, K_FULL = 1, K_EMPTY = 3, V_FULL = 5, V_EMPTY = 7, S_FULL = 9, P_FULL = 11,
@@ -61,7 +63,8 @@ struct Layout {
   static constexpr int OFF_MISC = OFF_BAR + 8 * NBAR;  // tmem holder, abort flag
   static constexpr int OFF_MASK = OFF_MISC + 16;
   static constexpr int OFF_VSC = OFF_MASK + 4 * kMaxW;  // per-channel output scales
-  static constexpr int BYTES = OFF_VSC + 4 * D;
+  static constexpr int OFF_XCH = OFF_VSC + 4 * D;       // row max / row sum exchange between halves
+  static constexpr int BYTES = OFF_XCH + 4 * 768;  // 256 maxima + 512 sums/maxima at the end
   // request at least 116 KB so that one CTA (and its 512 TMEM columns) owns an SM
   static constexpr int DYN = (BYTES + 1024 > 116 * 1024) ? BYTES + 1024 : 116 * 1024;
   // TMEM columns
@@ -86,7 +89,7 @@ __device__ __forceinline__ void raise_error(volatile int* abort, uint32_t code) 
   atomicOr(&g_attn_error_word, code);
 }
 
-template <int D>
+template <int D, int NPOLY>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_qfp4, const __grid_constant__ CUtensorMap tm_kfp4,
                     const __grid_constant__ CUtensorMap tm_qbf, const __grid_constant__ CUtensorMap tm_kbf,
@@ -118,7 +121,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     *abort = 0;
     fence_mbar_init();
   }
-  if (warp == 5) {
+  if (warp == 9) {
     tmem_alloc(smem_u32(tmem_holder), 512);
     tmem_relinquish();
   }
@@ -131,7 +134,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto is_hi = [&](int j) -> bool { return (mrow[j >> 5] >> (j & 31)) & 1u; };
   volatile int never = 0;
 
-  if (warp == 4) {
+  if (warp == 8) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       prefetch_tmap(&tm_qfp4); prefetch_tmap(&tm_kfp4); prefetch_tmap(&tm_qbf);
@@ -179,7 +182,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
       }
     }
-  } else if (warp == 5) {
+  } else if (warp == 9) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr int KB = D / 64;
@@ -255,71 +258,123 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ softmax
-    const int r = tid;  // query row within the tile == TMEM lane
-    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    // Two warpgroups take alternating key tiles: group w handles j = w, w+2, ...
+    // (S buffer w); each thread owns one full query row (= TMEM lane) of its
+    // tiles.  Only the exact running maximum is sequential across tiles: group
+    // w publishes m_j per row in shared memory (named-barrier arrive) and the
+    // other group waits for it (named-barrier sync) before its exponentials, so
+    // one group's exponentials overlap the other's loads, maxima and stores.
+    // Each group keeps its own partial row sum relative to the maximum of its
+    // own last tile; the two are combined at the end.
+    const int q4 = warp & 3, wg = warp >> 2;
+    const int r = q4 * 32 + lane;  // query row within the tile == TMEM lane
+    const uint32_t lane_base = (uint32_t)(q4 * 32) << 16;
     const int row_g = i * 128 + r;
+    float* mbuf = reinterpret_cast<float*>(smem + L::OFF_XCH);  // [2 groups][128 rows] running max
+    const uint32_t bar_out = 1 + wg * 4 + q4, bar_in = 1 + (wg ^ 1) * 4 + q4;
     const float sc_hi = p.scale_log2;
     const float sc_lo = p.scale_log2 * (p.q_gs[bhq] * p.k_gs[bhk]);
-    float m = -INFINITY, l = 0.0f;
+    float l = 0.0f, m_ref = -INFINITY;
     bool ok = true;
-    for (int j = 0; j < nj; ++j) {
-      const int s = j & 1, u = j >> 1;
+    for (int j = wg; j < nj; j += 2) {
+      const int u = j >> 1;
       const bool hi = is_hi(j);
-      if (!__all_sync(0xffffffffu, mbar_wait(BAR(S_FULL + s), u & 1, abort, kWaitLimitNs))) {
+      if (!__all_sync(0xffffffffu, mbar_wait(BAR(S_FULL + wg), u & 1, abort, kWaitLimitNs))) {
         raise_error(abort, 4u);
         ok = false;
         break;
       }
       tc_fence_after();
-      const uint32_t s_addr = tmem + lane_base + L::S_COL0 + 128 * s;
-      uint32_t sv[4][32];
+      const uint32_t s_addr = tmem + lane_base + L::S_COL0 + 128 * wg;
+      const bool edge = (p.causal && j == i) || ((j + 1) * 128 > p.N);  // warp-uniform
+      const int lim = min(p.causal ? row_g + 1 : p.N, p.N) - j * 128;    // columns >= lim are masked
+      // pass 1: row max of the raw logits (tree of three-input maxima)
+      float mloc;
+      {
+        uint32_t v[128];
 #pragma unroll
-      for (int c4 = 0; c4 < 4; ++c4) tmem_ld32(s_addr + 32 * c4, sv[c4]);
-      tmem_ld_wait();
-      const float sc = hi ? sc_hi : sc_lo;
-      const bool edge = (p.causal && j == i) || ((j + 1) * 128 > p.N);
-      const int lim = min(p.causal ? row_g + 1 : p.N, p.N) - j * 128;  // columns < lim are valid
-      float mx = -INFINITY;
+        for (int c4 = 0; c4 < 4; ++c4) tmem_ld32(s_addr + 32 * c4, *reinterpret_cast<uint32_t(*)[32]>(&v[32 * c4]));
+        tmem_ld_wait();
+        if (edge) {
 #pragma unroll
-      for (int c4 = 0; c4 < 4; ++c4)
-#pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          float x = __uint_as_float(sv[c4][c]);
-          if (edge && (c4 * 32 + c) >= lim) x = -INFINITY;
-          sv[c4][c] = __float_as_uint(x);
-          mx = fmaxf(mx, x);
+          for (int c = 0; c < 128; ++c)
+            if (c >= lim) v[c] = __float_as_uint(-INFINITY);
         }
-      const float m_new = fmaxf(m, mx * sc);
-      const float alpha = (m == -INFINITY) ? 0.0f : ex2_approx(m - m_new);
-      const float nb = 8.0f - m_new;  // p * 2^8 = 2^(s * sc - m_new + 8)
-      float rs = 0.0f;
-      uint32_t pa[32], pb[32];  // packed P: e4m3 uses pa (32 columns), bf16 uses pa then pb
-      if (hi) {
+        float t1[43];
 #pragma unroll
-        for (int c4 = 0; c4 < 4; ++c4)
+        for (int c = 0; c < 42; ++c)
+          t1[c] = fmax3(__uint_as_float(v[3 * c]), __uint_as_float(v[3 * c + 1]), __uint_as_float(v[3 * c + 2]));
+        t1[42] = fmaxf(__uint_as_float(v[126]), __uint_as_float(v[127]));
+        float t2[15];
 #pragma unroll
-          for (int c = 0; c < 32; c += 2) {
-            const float p0 = ex2_approx(fmaf(__uint_as_float(sv[c4][c]), sc, nb));
-            const float p1 = ex2_approx(fmaf(__uint_as_float(sv[c4][c + 1]), sc, nb));
-            rs += p0 + p1;
-            if (c4 < 2) pa[(c4 * 32 + c) >> 1] = cvt_bf16x2(p0, p1);
-            else pb[((c4 - 2) * 32 + c) >> 1] = cvt_bf16x2(p0, p1);
-          }
-      } else {
+        for (int c = 0; c < 14; ++c) t2[c] = fmax3(t1[3 * c], t1[3 * c + 1], t1[3 * c + 2]);
+        t2[14] = t1[42];
+        float t3[5];
 #pragma unroll
-        for (int c4 = 0; c4 < 4; ++c4)
-#pragma unroll
-          for (int c = 0; c < 32; c += 4) {
-            const float p0 = ex2_approx(fmaf(__uint_as_float(sv[c4][c]), sc, nb));
-            const float p1 = ex2_approx(fmaf(__uint_as_float(sv[c4][c + 1]), sc, nb));
-            const float p2 = ex2_approx(fmaf(__uint_as_float(sv[c4][c + 2]), sc, nb));
-            const float p3 = ex2_approx(fmaf(__uint_as_float(sv[c4][c + 3]), sc, nb));
-            rs += (p0 + p1) + (p2 + p3);
-            pa[(c4 * 32 + c) >> 2] = cvt_e4m3x2(p0, p1) | (cvt_e4m3x2(p2, p3) << 16);
-          }
+        for (int c = 0; c < 5; ++c) t3[c] = fmax3(t2[3 * c], t2[3 * c + 1], t2[3 * c + 2]);
+        mloc = fmaxf(fmax3(t3[0], t3[1], t3[2]), fmaxf(t3[3], t3[4]));
       }
-      l = l * alpha + rs;
-      // rescale O when any row of this warp has a new maximum (alpha == 1 is a no-op)
+      const float sc = hi ? sc_hi : sc_lo;
+      float m_prev = -INFINITY;
+      if (j > 0) {
+        named_bar_sync(bar_in, 64);
+        m_prev = mbuf[(wg ^ 1) * 128 + r];
+      }
+      const float m_new = fmaxf(m_prev, mloc * sc);
+      mbuf[wg * 128 + r] = m_new;
+      if (j + 1 < nj) named_bar_arrive(bar_out, 64);
+      const float alpha = (m_prev == -INFINITY) ? 0.0f : ex2_approx(m_prev - m_new);  // O rescale
+      const float beta = (m_ref == -INFINITY) ? 0.0f : ex2_approx(m_ref - m_new);     // own partial sum
+      const uint64_t sc2 = f2pack(sc, sc);
+      const uint64_t nb2 = f2pack(8.0f - m_new, 8.0f - m_new);  // p * 2^8 = 2^(s*sc - m_new + 8)
+      uint64_t acc[4] = {0, 0, 0, 0};
+      // pass 2: exponentials by halves of 64 columns, re-read from TMEM
+#pragma unroll
+      for (int h2 = 0; h2 < 2; ++h2) {
+        uint32_t v[64];
+        tmem_ld32(s_addr + 64 * h2, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
+        tmem_ld32(s_addr + 64 * h2 + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
+        tmem_ld_wait();
+        if (edge) {
+#pragma unroll
+          for (int c = 0; c < 64; ++c)
+            if (64 * h2 + c >= lim) v[c] = __float_as_uint(-INFINITY);
+        }
+        uint32_t pw[32];
+#pragma unroll
+        for (int t = 0; t < 32; ++t) {  // element pairs
+          const uint64_t a2 = ffma2(f2pack(__uint_as_float(v[2 * t]), __uint_as_float(v[2 * t + 1])), sc2, nb2);
+          uint64_t e2;
+          if ((t & 3) < NPOLY) {
+            e2 = exp2_poly2(a2);
+          } else {
+            float a0, a1;
+            f2unpack(a2, a0, a1);
+            e2 = f2pack(ex2_approx(a0), ex2_approx(a1));
+          }
+          acc[t & 3] = fadd2(acc[t & 3], e2);
+          float e0, e1;
+          f2unpack(e2, e0, e1);
+          if (hi) {
+            pw[t] = cvt_bf16x2(e0, e1);
+          } else {
+            const uint32_t hh = cvt_e4m3x2(e0, e1);
+            if (t & 1) pw[t >> 1] = __byte_perm(pw[t >> 1], hh, 0x5410);
+            else pw[t >> 1] = hh;
+          }
+        }
+        // P overwrites the leading columns of this S buffer (those logits are already consumed)
+        if (hi) tmem_st32(s_addr + 32 * h2, pw);
+        else tmem_st16(s_addr + 16 * h2, *reinterpret_cast<uint32_t(*)[16]>(&pw[0]));
+      }
+      float r0, r1, r2, r3, r4, r5, r6, r7;
+      f2unpack(acc[0], r0, r1);
+      f2unpack(acc[1], r2, r3);
+      f2unpack(acc[2], r4, r5);
+      f2unpack(acc[3], r6, r7);
+      l = l * beta + (((r0 + r1) + (r2 + r3)) + ((r4 + r5) + (r6 + r7)));
+      m_ref = m_new;
+      // rescale O when any row of the warp has a new maximum (alpha == 1 is a no-op)
       const bool corr = (j > 0) && (alpha != 1.0f);
       if (__any_sync(0xffffffffu, corr)) {
         if (!__all_sync(0xffffffffu, mbar_wait(BAR(PV_DONE), (j - 1) & 1, abort, kWaitLimitNs))) {
@@ -328,6 +383,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         tc_fence_after();
+        const uint64_t al2 = f2pack(alpha, alpha);
 #pragma unroll
         for (int c4 = 0; c4 < D / 32; ++c4) {
           uint32_t ov[32];
@@ -335,35 +391,46 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_ld32(o_addr, ov);
           tmem_ld_wait();
 #pragma unroll
-          for (int c = 0; c < 32; ++c) ov[c] = __float_as_uint(__uint_as_float(ov[c]) * alpha);
+          for (int c = 0; c < 32; c += 2) {
+            float a0, a1;
+            f2unpack(fmul2(f2pack(__uint_as_float(ov[c]), __uint_as_float(ov[c + 1])), al2), a0, a1);
+            ov[c] = __float_as_uint(a0);
+            ov[c + 1] = __float_as_uint(a1);
+          }
           tmem_st32(o_addr, ov);
         }
       }
-      // P overwrites the first columns of this S buffer
-      tmem_st32(s_addr, pa);
-      if (hi) tmem_st32(s_addr + 32, pb);
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(BAR(P_FULL + s));
-      m = m_new;
+      if (lane == 0) mbar_arrive(BAR(P_FULL + wg));
     }
     // ---------------------------------------------------------- epilogue
+    // combine the two groups' partial row sums, then each group writes D/2 columns
     ok = ok && __all_sync(0xffffffffu, mbar_wait(BAR(O_FINAL), 0, abort, kWaitLimitNs));
+    float* xl = reinterpret_cast<float*>(smem + L::OFF_XCH) + 256;  // [2][128] sums, [2][128] maxima
+    xl[wg * 128 + r] = l;
+    xl[256 + wg * 128 + r] = m_ref;
+    named_bar_sync(9 + q4, 64);
     if (ok) {
       tc_fence_after();
-      const float inv_l = 1.0f / l;
-      __nv_bfloat16* orow = p.o + ((size_t)bhq * p.N + row_g) * D;
+      const float lo_ = xl[(wg ^ 1) * 128 + r], mo_ = xl[256 + (wg ^ 1) * 128 + r];
+      const float m_fin = fmaxf(m_ref, mo_);
+      const float lt = (m_ref == -INFINITY ? 0.0f : l * ex2_approx(m_ref - m_fin)) +
+                       (mo_ == -INFINITY ? 0.0f : lo_ * ex2_approx(mo_ - m_fin));
+      const float inv_l = 1.0f / lt;
+      __nv_bfloat16* orow = p.o + ((size_t)bhq * p.N + row_g) * D + (D / 2) * wg;
 #pragma unroll
-      for (int c4 = 0; c4 < D / 32; ++c4) {
+      for (int c4 = 0; c4 < D / 64; ++c4) {
         uint32_t ov[32];
-        tmem_ld32(tmem + lane_base + L::O_COL + 32 * c4, ov);
+        tmem_ld32(tmem + lane_base + L::O_COL + (D / 2) * wg + 32 * c4, ov);
         tmem_ld_wait();
         uint32_t packed[16];
 #pragma unroll
         for (int c = 0; c < 32; c += 2) {
-          const float a0 = __uint_as_float(ov[c]) * (vsc[c4 * 32 + c] * inv_l);
-          const float a1 = __uint_as_float(ov[c + 1]) * (vsc[c4 * 32 + c + 1] * inv_l);
+          const int cc = (D / 2) * wg + c4 * 32 + c;
+          const float a0 = __uint_as_float(ov[c]) * (vsc[cc] * inv_l);
+          const float a1 = __uint_as_float(ov[c + 1]) * (vsc[cc + 1] * inv_l);
           packed[c >> 1] = cvt_bf16x2(a0, a1);
         }
         if (row_g < p.N) {
@@ -373,8 +440,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             dst[q] = make_uint4(packed[4 * q], packed[4 * q + 1], packed[4 * q + 2], packed[4 * q + 3]);
         }
       }
-      if (p.lse != nullptr && row_g < p.N)
-        p.lse[(size_t)bhq * p.N + row_g] = (m - 8.0f) * 0.69314718055994531f + logf(l);
+      if (wg == 0 && p.lse != nullptr && row_g < p.N)
+        p.lse[(size_t)bhq * p.N + row_g] = (m_fin - 8.0f) * 0.69314718055994531f + logf(lt);
     } else {
       raise_error(abort, 4u);
     }
@@ -383,7 +450,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // ------------------------------------------------------------ teardown
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == 9) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
@@ -422,6 +489,18 @@ static bool make_map(CUtensorMap* m, CUtensorMapDataType dt, const void* base, u
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Share of exponentials computed by the FMA-pipe polynomial instead of the MUFU
+// unit: npoly of every 4 element pairs.  Tunable with THRIFT_EXP_POLY (0..2).
+static int exp_poly_pairs() {
+  static int v = -1;
+  if (v < 0) {
+    const char* e = getenv("THRIFT_EXP_POLY");
+    int x = e ? atoi(e) : kDefaultPolyPairs;
+    v = x < 0 ? 0 : (x > 2 ? 2 : x);
+  }
+  return v;
+}
+
 template <int D>
 static int launch_d(const AttnArgs& a, cudaStream_t st) {
   using L = Layout<D>;
@@ -455,10 +534,16 @@ static int launch_d(const AttnArgs& a, cudaStream_t st) {
   p.B = a.B; p.Hq = a.Hq; p.Hkv = a.Hkv; p.N = a.N; p.T = T; p.W = W; p.causal = a.causal;
   const float scale = a.softmax_scale > 0.0f ? a.softmax_scale : 1.0f / sqrtf((float)D);
   p.scale_log2 = scale * 1.4426950408889634f;
-  if (cudaFuncSetAttribute(attn_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::DYN) != cudaSuccess)
+  auto kern = attn_fwd_kernel<D, 0>;
+  switch (exp_poly_pairs()) {
+    case 1: kern = attn_fwd_kernel<D, 1>; break;
+    case 2: kern = attn_fwd_kernel<D, 2>; break;
+    default: break;
+  }
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::DYN) != cudaSuccess)
     return THRIFT_ERR_CUDA;
   const unsigned grid = (unsigned)(BHq * (uint64_t)T);
-  attn_fwd_kernel<D><<<grid, kThreads, L::DYN, st>>>(m_qfp4, m_kfp4, m_qbf, m_kbf, m_vfp8, m_vbf, p);
+  kern<<<grid, kThreads, L::DYN, st>>>(m_qfp4, m_kfp4, m_qbf, m_kbf, m_vfp8, m_vbf, p);
   count_launches(1);
   return cudaGetLastError() == cudaSuccess ? THRIFT_OK : THRIFT_ERR_CUDA;
 }

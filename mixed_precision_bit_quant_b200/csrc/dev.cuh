@@ -253,6 +253,94 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};"
+      ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]),
+        "r"(r[7]), "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+        "r"(r[15])
+      : "memory");
+}
+
+// Producer side of a named barrier: arrive without waiting.
+__device__ __forceinline__ void named_bar_arrive(uint32_t id, uint32_t count) {
+  asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
+// Named barrier over `count` threads (ids 1..15; id 0 is __syncthreads).
+__device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
+// ---------------------------------------------------------------------------
+// Packed FP32x2 arithmetic (one instruction, two lanes of a 64-bit register pair).
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint64_t f2pack(float a, float b) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ void f2unpack(uint64_t r, float& a, float& b) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(r));
+}
+__device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t fadd2_rm(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rm.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t fmul2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// 2^x for two arguments on the FMA pipe (x <= 128).  x is clamped to >= -127;
+// n = floor(x) by adding 1.5 * 2^23 with round-toward-minus-infinity, f = x - n in
+// [0, 1) exactly, 2^f by a degree-4 polynomial (coefficients fitted here by
+// relative-error least squares on [0, 1): max relative error 2.7e-6 in FP32),
+// and n is added to the exponent field of the result.
+__device__ __forceinline__ uint64_t exp2_poly2(uint64_t x2) {
+  float x0, x1;
+  f2unpack(x2, x0, x1);
+  x0 = fmaxf(x0, -127.0f);
+  x1 = fmaxf(x1, -127.0f);
+  x2 = f2pack(x0, x1);
+  const uint64_t C = f2pack(12582912.0f, 12582912.0f);
+  const uint64_t t2 = fadd2_rm(x2, C);                       // 1.5*2^23 + floor(x)
+  const uint64_t nC = f2pack(-12582912.0f, -12582912.0f);
+  const uint64_t n2 = fadd2(t2, nC);                          // floor(x), exact
+  float n0, n1;
+  f2unpack(n2, n0, n1);
+  const uint64_t f2 = fadd2(x2, f2pack(-n0, -n1));            // x - floor(x), exact
+  uint64_t p = f2pack(1.3534157536923885e-2f, 1.3534157536923885e-2f);
+  p = ffma2(p, f2, f2pack(5.2011482417583466e-2f, 5.2011482417583466e-2f));
+  p = ffma2(p, f2, f2pack(2.414427399635315e-1f, 2.414427399635315e-1f));
+  p = ffma2(p, f2, f2pack(6.930038332939148e-1f, 6.930038332939148e-1f));
+  p = ffma2(p, f2, f2pack(1.0000026226043701f, 1.0000026226043701f));
+  float p0, p1, t0, t1;
+  f2unpack(p, p0, p1);
+  f2unpack(t2, t0, t1);
+  const float r0 = __uint_as_float(__float_as_uint(p0) + (__float_as_uint(t0) << 23));
+  const float r1 = __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23));
+  return f2pack(r0, r1);
+}
+
 // ---------------------------------------------------------------------------
 // Conversions for P.
 // ---------------------------------------------------------------------------
