@@ -7,21 +7,26 @@
 // (abstract): one hybrid-precision attention operator for prefill.
 //
 // One CTA computes one 128-row query tile (b, hq, i) against the key tiles
-// j = 0 .. (causal ? i : T-1) in ascending order.  Warp roles:
-//   warps 0-3  softmax: one thread per query row (= TMEM lane); reads S from
-//              TMEM, masks, exact running max, exp2, row sums, writes P back
-//              into TMEM (e4m3 or bf16), rescales O in TMEM when the row max
-//              grows, final epilogue O * 2^e_c / l -> bf16.
-//   warp 4     TMA producer: Q (NVFP4 + scales + BF16) once, then per key
-//              tile either NVFP4 K + scales and e4m3 V^T, or BF16 K and V^T,
-//              following the tile's mask bit; two stages each.
-//   warp 5     TMEM allocator and MMA issuer (one thread):
-//              FP4 pair: S = Q4 K4^T  kind::mxf4nvf4 (block scales in TMEM)
-//                        O += P8 V8   kind::f8f6f4, P read from TMEM
-//              BF16 pair: S = Q K^T   kind::f16
-//                        O += P16 Vs  kind::f16, P read from TMEM
-// TMEM columns: S double buffer [0,256), O [256, 256+D), scale factors after.
-// The S computation of tile j+1 overlaps the softmax of tile j.
+// j = 0 .. (causal ? i : T-1) in ascending order.  384 threads, 12 warps:
+//   warps 0-3 / 4-7  softmax groups 0 / 1; group w takes tiles j = w, w+2, ...
+//              One thread owns one query row (= TMEM lane) of its tiles: read S
+//              from TMEM once, mask edge tiles, row max, take the exact running
+//              maximum from the other group (shared memory + mbarrier), exp2,
+//              partial row sums, P (e4m3 or bf16) into TMEM, O rescaled in TMEM
+//              when a row's maximum grows.
+//   warps 8/10 TMA producers: warp 8 loads Q (NVFP4 + scales + BF16) once and
+//              per key tile NVFP4 K + scales or BF16 K; warp 10 loads e4m3 V^T or
+//              BF16 V^T, per mask bit.
+//   warp 9     TMEM allocator and QK^T issuer (one thread): FP4 pair
+//              S = Q4 K4^T kind::mxf4nvf4 (block scales in TMEM), BF16 pair
+//              S = Q K^T kind::f16; S of tile j+2 as soon as group j%2 read S_j.
+//   warp 11    P.V issuer (one thread): O += P8 V8 kind::f8f6f4 or O += P16 Vs
+//              kind::f16, P read from TMEM; publishes the count of completed
+//              products in shared memory (the only P.V progress signal).
+//   Warps 8-11 form the third warpgroup, whose registers the softmax warps
+//   take over with setmaxnreg.
+// TMEM columns: S double buffer [0,256), O [256,256+D), three 32-column e4m3 P
+// regions [256+D, 352+D) (BF16 tiles keep P in their S buffer), block scales after.
 #include <cuda.h>
 #include <stdlib.h>
 
@@ -35,13 +40,23 @@ __device__ uint32_t g_attn_error_word;
 namespace attn {
 
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s per wait: far above any legitimate wait
-constexpr int kThreads = 320;  // 8 softmax warps, 1 TMA warp, 1 MMA warp
+constexpr int kThreads = 384;                       // 8 softmax warps + 4 producer / issuer warps
+constexpr int kSoftmaxRegs = 224, kOtherRegs = 56;  // 256*224 + 128*56 = 384*168 (the launch budget)
 constexpr int kMaxW = 128;                          // mask words per query tile (T <= 4096)
 constexpr int kDefaultPolyPairs = 0;
 
+// Operand rings: FP4 tiles use NLO slots of K (e2m1 + scales) and of V^T (e4m3);
+// BF16 tiles use NHI slots of bf16 K and V^T.  Producer and MMA issuer walk the
+// tiles in order and count FP4 and BF16 tiles separately to find slot and phase.
+constexpr int NLO = 4, NHI = 1;
 enum Bar : int {
-  Q_FULL = 0, K_FULL = 1, K_EMPTY = 3, V_FULL = 5, V_EMPTY = 7, S_FULL = 9, P_FULL = 11,
-  PV_DONE = 13, O_FINAL = 14, DRAIN = 15, NBAR = 16
+  Q_FULL = 0,
+  KL_FULL = 1, KL_EMPTY = KL_FULL + NLO, VL_FULL = KL_EMPTY + NLO, VL_EMPTY = VL_FULL + NLO,
+  KH_FULL = VL_EMPTY + NLO, KH_EMPTY = KH_FULL + NHI, VH_FULL = KH_EMPTY + NHI, VH_EMPTY = VH_FULL + NHI,
+  S_FULL = VH_EMPTY + NHI, S_FREE = S_FULL + 2, P_FULL = S_FREE + 2, PVC = P_FULL + 2,
+  QK_DRAIN = PVC + 2, PV_DRAIN = QK_DRAIN + 1,
+  MX = PV_DRAIN + 1,  // running-max hand-off [group][quarter]
+  NBAR = MX + 8
 };
 
 __host__ __device__ constexpr int al(int x, int a) { return (x + a - 1) / a * a; }
@@ -51,24 +66,32 @@ struct Layout {
   static constexpr int QFP4 = 128 * D / 2;    // packed e2m1 Q tile
   static constexpr int QBF = 128 * D * 2;      // bf16 Q tile (D/64 boxes of 128 x 64)
   static constexpr int SF = (D / 64) * 512;    // block scales of one tile, tensor-core order
-  static constexpr int KBUF = 128 * D * 2;     // max(e2m1 K tile, bf16 K tile)
-  static constexpr int VBUF = D * 128 * 2;     // max(e4m3 V^T tile, bf16 V^T tile)
+  static constexpr int KLO = 128 * D / 2;     // e2m1 K tile
+  static constexpr int VLO = D * 128;         // e4m3 V^T tile
+  static constexpr int KHI = 128 * D * 2;     // bf16 K tile (D/64 boxes of 128 x 64)
+  static constexpr int VHI = D * 128 * 2;     // bf16 V^T tile (2 boxes of D x 64)
   static constexpr int OFF_QFP4 = 0;
   static constexpr int OFF_QBF = al(OFF_QFP4 + QFP4, 1024);
-  static constexpr int OFF_K = OFF_QBF + QBF;          // two stages
-  static constexpr int OFF_V = OFF_K + 2 * KBUF;       // two stages
-  static constexpr int OFF_QSF = OFF_V + 2 * VBUF;
-  static constexpr int OFF_KSF = OFF_QSF + SF;         // two stages
-  static constexpr int OFF_BAR = al(OFF_KSF + 2 * SF, 64);
-  static constexpr int OFF_MISC = OFF_BAR + 8 * NBAR;  // tmem holder, abort flag
-  static constexpr int OFF_MASK = OFF_MISC + 16;
+  static constexpr int OFF_KL = OFF_QBF + QBF;         // NLO slots
+  static constexpr int OFF_VL = OFF_KL + NLO * KLO;    // NLO slots
+  static constexpr int OFF_KH = OFF_VL + NLO * VLO;    // NHI slots
+  static constexpr int OFF_VH = OFF_KH + NHI * KHI;    // NHI slots
+  static constexpr int OFF_QSF = OFF_VH + NHI * VHI;
+  static constexpr int OFF_KSF = OFF_QSF + SF;         // NLO slots
+  static constexpr int OFF_BAR = al(OFF_KSF + NLO * SF, 64);
+  static constexpr int OFF_MISC = OFF_BAR + 8 * NBAR;  // tmem holder, abort flag, completed-P.V count
+  static constexpr int OFF_MASK = al(OFF_MISC + 16, 16);
   static constexpr int OFF_VSC = OFF_MASK + 4 * kMaxW;  // per-channel output scales
-  static constexpr int OFF_XCH = OFF_VSC + 4 * D;       // row max / row sum exchange between halves
-  static constexpr int BYTES = OFF_XCH + 4 * 768;  // 256 maxima + 512 sums/maxima at the end
+  static constexpr int OFF_XCH = OFF_VSC + 4 * D;       // running maxima [2 groups][128 rows]
+  static constexpr int OFF_FIN = OFF_XCH + 4 * 256;     // final partial sums [2][128], maxima [2][128]
+  static constexpr int BYTES = OFF_FIN + 4 * 512;
   // request at least 116 KB so that one CTA (and its 512 TMEM columns) owns an SM
   static constexpr int DYN = (BYTES + 1024 > 116 * 1024) ? BYTES + 1024 : 116 * 1024;
   // TMEM columns
-  static constexpr uint32_t S_COL0 = 0, O_COL = 256, SFA_COL = 256 + D, SFB_COL0 = SFA_COL + 8;
+  // FP4 tiles write P (e4m3, 32 columns) into P region j % 3; BF16 tiles write P
+  // (bf16, 64 columns) over the leading columns of their own S buffer.
+  static constexpr uint32_t S_COL0 = 0, O_COL = 256, P_COL = 256 + D, SFA_COL = P_COL + 96,
+                            SFB_COL0 = SFA_COL + 8;
 };
 
 struct Params {
@@ -117,8 +140,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   float* vsc = reinterpret_cast<float*>(smem + L::OFF_VSC);
 
   if (tid == 0) {
-    for (int k = 0; k < NBAR; ++k) mbar_init(BAR(k), (k == P_FULL || k == P_FULL + 1) ? 4 : 1);
+    for (int k = 0; k < NBAR; ++k) {
+      const bool by_group = (k >= S_FREE && k < S_FREE + 2) || (k >= P_FULL && k < P_FULL + 2);
+      mbar_init(BAR(k), by_group ? 4 : 1);  // softmax barriers: one arrival per warp of the group
+    }
     *abort = 0;
+    *reinterpret_cast<volatile uint32_t*>(smem + L::OFF_MISC + 8) = 0u;
     fence_mbar_init();
   }
   if (warp == 9) {
@@ -133,173 +160,229 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = *tmem_holder;
   auto is_hi = [&](int j) -> bool { return (mrow[j >> 5] >> (j & 31)) & 1u; };
   volatile int never = 0;
+  const uint32_t pv_count = sb + L::OFF_MISC + 8;  // number of completed P.V products, in tile order
 
-  if (warp == 8) {
-    // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      prefetch_tmap(&tm_qfp4); prefetch_tmap(&tm_kfp4); prefetch_tmap(&tm_qbf);
-      prefetch_tmap(&tm_kbf); prefetch_tmap(&tm_vfp8); prefetch_tmap(&tm_vbf);
-      mbar_expect_tx(BAR(Q_FULL), L::QFP4 + L::QBF + L::SF);
-      tma_load_3d(sb + L::OFF_QFP4, &tm_qfp4, 0, i * 128, bhq, BAR(Q_FULL));
-      tma_load_3d(sb + L::OFF_QBF, &tm_qbf, 0, i * 128, bhq, BAR(Q_FULL));
-      if (D == 128) tma_load_3d(sb + L::OFF_QBF + 16384, &tm_qbf, 64, i * 128, bhq, BAR(Q_FULL));
-      bulk_load(sb + L::OFF_QSF, p.q_sf_mma + ((size_t)bhq * p.T + i) * L::SF, L::SF, BAR(Q_FULL));
-      int fills[2] = {0, 0};
+  if (warp >= 8) {
+    regs_dec<kOtherRegs>();
+    if ((warp == 8 || warp == 10) && lane == 0) {
+      // ---------------------------------------------------------- producers
+      // warp 8 loads Q once and the K tiles, warp 10 the V tiles: K loads run
+      // ahead of the softmax, bounded only by the QK^T that frees their stage.
+      const bool kside = (warp == 8);
+      if (kside) {
+        prefetch_tmap(&tm_qfp4); prefetch_tmap(&tm_kfp4); prefetch_tmap(&tm_qbf); prefetch_tmap(&tm_kbf);
+        mbar_expect_tx(BAR(Q_FULL), L::QFP4 + L::QBF + L::SF);
+        tma_load_3d(sb + L::OFF_QFP4, &tm_qfp4, 0, i * 128, bhq, BAR(Q_FULL));
+        tma_load_3d(sb + L::OFF_QBF, &tm_qbf, 0, i * 128, bhq, BAR(Q_FULL));
+        if (D == 128) tma_load_3d(sb + L::OFF_QBF + 16384, &tm_qbf, 64, i * 128, bhq, BAR(Q_FULL));
+        bulk_load(sb + L::OFF_QSF, p.q_sf_mma + ((size_t)bhq * p.T + i) * L::SF, L::SF, BAR(Q_FULL));
+      } else {
+        prefetch_tmap(&tm_vfp8); prefetch_tmap(&tm_vbf);
+      }
+      int nlo = 0, nhi = 0;
       for (int j = 0; j < nj; ++j) {
-        const int s = j & 1, u = j >> 1;
         const bool hi = is_hi(j);
-        const uint32_t kb = sb + L::OFF_K + s * L::KBUF;
-        const uint32_t vb = sb + L::OFF_V + s * L::VBUF;
-        if (u > 0 && !mbar_wait(BAR(K_EMPTY + s), (u - 1) & 1, abort, kWaitLimitNs)) { raise_error(abort, 1u); break; }
-        if (hi) {
-          mbar_expect_tx(BAR(K_FULL + s), 128 * D * 2);
-          tma_load_3d(kb, &tm_kbf, 0, j * 128, bhk, BAR(K_FULL + s));
-          if (D == 128) tma_load_3d(kb + 16384, &tm_kbf, 64, j * 128, bhk, BAR(K_FULL + s));
-        } else {
-          mbar_expect_tx(BAR(K_FULL + s), L::QFP4 + L::SF);
-          tma_load_3d(kb, &tm_kfp4, 0, j * 128, bhk, BAR(K_FULL + s));
-          bulk_load(sb + L::OFF_KSF + s * L::SF, p.k_sf_mma + ((size_t)bhk * p.T + j) * L::SF, L::SF,
-                    BAR(K_FULL + s));
+        const int n = hi ? nhi : nlo, slots = hi ? NHI : NLO, slot = n % slots, use = n / slots;
+        const int FULL = kside ? (hi ? KH_FULL : KL_FULL) : (hi ? VH_FULL : VL_FULL);
+        const int EMPTY = kside ? (hi ? KH_EMPTY : KL_EMPTY) : (hi ? VH_EMPTY : VL_EMPTY);
+        if (use > 0 && !mbar_wait(BAR(EMPTY + slot), (use - 1) & 1, abort, kWaitLimitNs)) {
+          raise_error(abort, 1u);
+          break;
         }
-        if (u > 0 && !mbar_wait(BAR(V_EMPTY + s), (u - 1) & 1, abort, kWaitLimitNs)) { raise_error(abort, 1u); break; }
-        if (hi) {
-          mbar_expect_tx(BAR(V_FULL + s), D * 128 * 2);
-          tma_load_3d(vb, &tm_vbf, j * 128, 0, bhk, BAR(V_FULL + s));
-          tma_load_3d(vb + D * 128, &tm_vbf, j * 128 + 64, 0, bhk, BAR(V_FULL + s));
+        const uint32_t full = BAR(FULL + slot);
+        if (kside) {
+          if (hi) {
+            const uint32_t kb = sb + L::OFF_KH + slot * L::KHI;
+            mbar_expect_tx(full, L::KHI);
+            tma_load_3d(kb, &tm_kbf, 0, j * 128, bhk, full);
+            if (D == 128) tma_load_3d(kb + 16384, &tm_kbf, 64, j * 128, bhk, full);
+          } else {
+            mbar_expect_tx(full, L::KLO + L::SF);
+            tma_load_3d(sb + L::OFF_KL + slot * L::KLO, &tm_kfp4, 0, j * 128, bhk, full);
+            bulk_load(sb + L::OFF_KSF + slot * L::SF, p.k_sf_mma + ((size_t)bhk * p.T + j) * L::SF, L::SF, full);
+          }
         } else {
-          mbar_expect_tx(BAR(V_FULL + s), D * 128);
-          tma_load_3d(vb, &tm_vfp8, j * 128, 0, bhk, BAR(V_FULL + s));
+          if (hi) {
+            const uint32_t vb = sb + L::OFF_VH + slot * L::VHI;
+            mbar_expect_tx(full, L::VHI);
+            tma_load_3d(vb, &tm_vbf, j * 128, 0, bhk, full);
+            tma_load_3d(vb + D * 128, &tm_vbf, j * 128 + 64, 0, bhk, full);
+          } else {
+            mbar_expect_tx(full, L::VLO);
+            tma_load_3d(sb + L::OFF_VL + slot * L::VLO, &tm_vfp8, j * 128, 0, bhk, full);
+          }
         }
-        fills[s] = u + 1;
+        if (hi) ++nhi; else ++nlo;
       }
       if (*abort) {
         // let copies already in flight land before the CTA's shared memory goes away
-        mbar_wait(BAR(Q_FULL), 0, &never, kWaitLimitNs / 4);
-        for (int s = 0; s < 2; ++s)
-          if (fills[s] > 0) {
-            mbar_wait(BAR(K_FULL + s), (fills[s] - 1) & 1, &never, kWaitLimitNs / 4);
-            mbar_wait(BAR(V_FULL + s), (fills[s] - 1) & 1, &never, kWaitLimitNs / 4);
-          }
+        if (kside) mbar_wait(BAR(Q_FULL), 0, &never, kWaitLimitNs / 4);
+        for (int k = 0; k < NLO && k < nlo; ++k) {
+          const int n = nlo - 1 - k, slot = n % NLO;
+          mbar_wait(BAR((kside ? KL_FULL : VL_FULL) + slot), (n / NLO) & 1, &never, kWaitLimitNs / 4);
+        }
+        for (int k = 0; k < NHI && k < nhi; ++k) {
+          const int n = nhi - 1 - k, slot = n % NHI;
+          mbar_wait(BAR((kside ? KH_FULL : VH_FULL) + slot), (n / NHI) & 1, &never, kWaitLimitNs / 4);
+        }
       }
-    }
-  } else if (warp == 9) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    } else if (warp == 9 && lane == 0) {
+      // ---------------------------------------------------------- QK^T issuer
       constexpr int KB = D / 64;
       constexpr uint32_t fp4_row = D / 2;
       constexpr uint32_t fp4_swz = (D == 128) ? SWZ_64B : SWZ_32B;
       bool ok = mbar_wait(BAR(Q_FULL), 0, abort, kWaitLimitNs);
-      if (!ok) raise_error(abort, 2u);
       if (ok) {
         tc_fence_after();
 #pragma unroll
         for (int kb = 0; kb < KB; ++kb)
           tmem_cp_32x128b_x4(tmem + L::SFA_COL + 4 * kb, smem_desc(sb + L::OFF_QSF + kb * 512, 16, 128, SWZ_NONE));
       }
-      for (int j = 0; ok && j <= nj; ++j) {
-        if (j < nj) {
-          const int s = j & 1, u = j >> 1;
-          if (!mbar_wait(BAR(K_FULL + s), u & 1, abort, kWaitLimitNs)) { raise_error(abort, 2u); ok = false; break; }
-          tc_fence_after();
-          const uint32_t d_s = tmem + L::S_COL0 + 128 * s;
-          const uint32_t kb_addr = sb + L::OFF_K + s * L::KBUF;
-          if (is_hi(j)) {
-#pragma unroll
-            for (int k = 0; k < D / 16; ++k) {
-              const uint32_t off = (k >> 2) * 16384 + (k & 3) * 32;
-              mma_bf16_ss(d_s, smem_desc(sb + L::OFF_QBF + off, 16, 1024, SWZ_128B),
-                          smem_desc(kb_addr + off, 16, 1024, SWZ_128B), idesc_bf16(128), k > 0);
-            }
-          } else {
-            const uint32_t sfb = tmem + L::SFB_COL0 + 8 * s;
-#pragma unroll
-            for (int kb = 0; kb < KB; ++kb)
-              tmem_cp_32x128b_x4(sfb + 4 * kb, smem_desc(sb + L::OFF_KSF + s * L::SF + kb * 512, 16, 128, SWZ_NONE));
-#pragma unroll
-            for (int kb = 0; kb < KB; ++kb)
-              mma_nvfp4_ss(d_s, smem_desc(sb + L::OFF_QFP4 + kb * 32, 16, 8 * fp4_row, fp4_swz),
-                           smem_desc(kb_addr + kb * 32, 16, 8 * fp4_row, fp4_swz), idesc_nvfp4(128),
-                           tmem + L::SFA_COL + 4 * kb, sfb + 4 * kb, kb > 0);
+      int n_lo = 0, n_hi = 0;
+      uint32_t mw = 0;
+      for (int j = 0; ok && j < nj; ++j) {
+        if ((j & 31) == 0) mw = mrow[j >> 5];
+        const bool hi = (mw >> (j & 31)) & 1u;
+        const int s = j & 1;
+        // S buffer s is free once the softmax group has read S_{j-2} and, when tile j-2 was
+        // BF16 (its P lives in that buffer), once P_{j-2} V_{j-2} has completed
+        if (j >= 2) {
+          if (!mbar_wait(BAR(S_FREE + s), ((j - 2) >> 1) & 1, abort, kWaitLimitNs)) { ok = false; break; }
+          if (((j - 2) >> 5) == (j >> 5) ? ((mw >> ((j - 2) & 31)) & 1u) : is_hi(j - 2)) {
+            if (!count_wait(pv_count, (uint32_t)(j - 1), abort, kWaitLimitNs)) { ok = false; break; }
           }
-          tc_commit(BAR(S_FULL + s));
-          tc_commit(BAR(K_EMPTY + s));
         }
-        if (j >= 1) {
-          const int jj = j - 1, s2 = jj & 1, u2 = jj >> 1;
-          if (!mbar_wait(BAR(P_FULL + s2), u2 & 1, abort, kWaitLimitNs) ||
-              !mbar_wait(BAR(V_FULL + s2), u2 & 1, abort, kWaitLimitNs)) {
-            raise_error(abort, 2u);
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t a_p = tmem + L::S_COL0 + 128 * s2;
-          const uint32_t vb = sb + L::OFF_V + s2 * L::VBUF;
-          const uint32_t d_o = tmem + L::O_COL;
-          if (is_hi(jj)) {
+        const int n = hi ? n_hi : n_lo, slots = hi ? NHI : NLO, slot = n % slots, use = n / slots;
+        if (!mbar_wait(BAR((hi ? KH_FULL : KL_FULL) + slot), use & 1, abort, kWaitLimitNs)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t d_s = tmem + L::S_COL0 + 128 * s;
+        if (hi) {
+          const uint32_t kb_addr = sb + L::OFF_KH + slot * L::KHI;
 #pragma unroll
-            for (int k = 0; k < 8; ++k)
-              mma_bf16_ts(d_o, a_p + 8 * k, smem_desc(vb + (k >> 2) * (D * 128) + (k & 3) * 32, 16, 1024, SWZ_128B),
-                          idesc_bf16(D), (jj > 0 || k > 0) ? 1u : 0u);
-          } else {
-#pragma unroll
-            for (int k = 0; k < 4; ++k)
-              mma_e4m3_ts(d_o, a_p + 8 * k, smem_desc(vb + k * 32, 16, 1024, SWZ_128B), idesc_e4m3(D),
-                          (jj > 0 || k > 0) ? 1u : 0u);
+          for (int k = 0; k < D / 16; ++k) {
+            const uint32_t off = (k >> 2) * 16384 + (k & 3) * 32;
+            mma_bf16_ss(d_s, smem_desc(sb + L::OFF_QBF + off, 16, 1024, SWZ_128B),
+                        smem_desc(kb_addr + off, 16, 1024, SWZ_128B), idesc_bf16(128), k > 0);
           }
-          tc_commit(BAR(V_EMPTY + s2));
-          tc_commit(BAR(PV_DONE));
-          if (jj == nj - 1) tc_commit(BAR(O_FINAL));
+          tc_commit(BAR(KH_EMPTY + slot));
+          ++n_hi;
+        } else {
+          const uint32_t kb_addr = sb + L::OFF_KL + slot * L::KLO;
+          const uint32_t sfb = tmem + L::SFB_COL0 + 8 * s;
+#pragma unroll
+          for (int kb = 0; kb < KB; ++kb)
+            tmem_cp_32x128b_x4(sfb + 4 * kb, smem_desc(sb + L::OFF_KSF + slot * L::SF + kb * 512, 16, 128, SWZ_NONE));
+#pragma unroll
+          for (int kb = 0; kb < KB; ++kb)
+            mma_nvfp4_ss(d_s, smem_desc(sb + L::OFF_QFP4 + kb * 32, 16, 8 * fp4_row, fp4_swz),
+                         smem_desc(kb_addr + kb * 32, 16, 8 * fp4_row, fp4_swz), idesc_nvfp4(128),
+                         tmem + L::SFA_COL + 4 * kb, sfb + 4 * kb, kb > 0);
+          tc_commit(BAR(KL_EMPTY + slot));
+          ++n_lo;
         }
+        tc_commit(BAR(S_FULL + s));
       }
+      if (!ok) raise_error(abort, 2u);
       // every tcgen05 op issued above completes before TMEM is released
-      tc_commit(BAR(DRAIN));
-      mbar_wait(BAR(DRAIN), 0, &never, kWaitLimitNs);
+      tc_commit(BAR(QK_DRAIN));
+      mbar_wait(BAR(QK_DRAIN), 0, &never, kWaitLimitNs);
+    } else if (warp == 11 && lane == 0) {
+      // ---------------------------------------------------------- P.V issuer
+      // Issues P_t V_t in order, waits for its completion and publishes the count of
+      // completed products, which the softmax groups and the epilogue wait on.
+      bool ok = true;
+      int n_lo = 0, n_hi = 0;
+      uint32_t mw = 0;
+      for (int t = 0; t < nj; ++t) {
+        if ((t & 31) == 0) mw = mrow[t >> 5];
+        const bool hi = (mw >> (t & 31)) & 1u;
+        const int s = t & 1, u = t >> 1;
+        const int n = hi ? n_hi : n_lo, slots = hi ? NHI : NLO, slot = n % slots, use = n / slots;
+        if (!mbar_wait(BAR(P_FULL + s), u & 1, abort, kWaitLimitNs) ||
+            !mbar_wait(BAR((hi ? VH_FULL : VL_FULL) + slot), use & 1, abort, kWaitLimitNs)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_o = tmem + L::O_COL;
+        if (hi) {
+          const uint32_t vb = sb + L::OFF_VH + slot * L::VHI;
+          const uint32_t a_p = tmem + L::S_COL0 + 128 * s;
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+            mma_bf16_ts(d_o, a_p + 8 * k, smem_desc(vb + (k >> 2) * (D * 128) + (k & 3) * 32, 16, 1024, SWZ_128B),
+                        idesc_bf16(D), (t > 0 || k > 0) ? 1u : 0u);
+          tc_commit(BAR(VH_EMPTY + slot));
+          ++n_hi;
+        } else {
+          const uint32_t vb = sb + L::OFF_VL + slot * L::VLO;
+          const uint32_t a_p = tmem + L::P_COL + 32 * (t % 3);
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            mma_e4m3_ts(d_o, a_p + 8 * k, smem_desc(vb + k * 32, 16, 1024, SWZ_128B), idesc_e4m3(D),
+                        (t > 0 || k > 0) ? 1u : 0u);
+          tc_commit(BAR(VL_EMPTY + slot));
+          ++n_lo;
+        }
+        tc_commit(BAR(PVC + s));
+        if (!mbar_wait(BAR(PVC + s), u & 1, abort, kWaitLimitNs)) { ok = false; break; }
+        tc_fence_after();
+        st_release_u32(pv_count, (uint32_t)(t + 1));
+      }
+      if (!ok) raise_error(abort, 2u);
+      tc_commit(BAR(PV_DRAIN));
+      mbar_wait(BAR(PV_DRAIN), 0, &never, kWaitLimitNs);
     }
   } else {
+    regs_inc<kSoftmaxRegs>();
     // ------------------------------------------------------------ softmax
-    // Two warpgroups take alternating key tiles: group w handles j = w, w+2, ...
-    // (S buffer w); each thread owns one full query row (= TMEM lane) of its
-    // tiles.  Only the exact running maximum is sequential across tiles: group
-    // w publishes m_j per row in shared memory (named-barrier arrive) and the
-    // other group waits for it (named-barrier sync) before its exponentials, so
-    // one group's exponentials overlap the other's loads, maxima and stores.
-    // Each group keeps its own partial row sum relative to the maximum of its
-    // own last tile; the two are combined at the end.
+    // Two groups of four warps: group wg takes the key tiles j = wg, wg+2, ... (S
+    // buffer wg) and each thread owns one query row (= TMEM lane).  The exact
+    // running maximum is the only sequential state across tiles: group wg writes
+    // m_j per row to shared memory and signals the other group (mbarrier) as soon
+    // as it is known, so one group's exponentials overlap the other group's loads,
+    // maxima, stores and O rescales.  Each group keeps its own partial row sum
+    // relative to the maximum of its own last tile; both are combined at the end.
     const int q4 = warp & 3, wg = warp >> 2;
     const int r = q4 * 32 + lane;  // query row within the tile == TMEM lane
     const uint32_t lane_base = (uint32_t)(q4 * 32) << 16;
     const int row_g = i * 128 + r;
     float* mbuf = reinterpret_cast<float*>(smem + L::OFF_XCH);  // [2 groups][128 rows] running max
-    const uint32_t bar_out = 1 + wg * 4 + q4, bar_in = 1 + (wg ^ 1) * 4 + q4;
+    const uint32_t mx_out = BAR(MX + wg * 4 + q4), mx_in = BAR(MX + (wg ^ 1) * 4 + q4);
     const float sc_hi = p.scale_log2;
     const float sc_lo = p.scale_log2 * (p.q_gs[bhq] * p.k_gs[bhk]);
+    const uint32_t p_base = tmem + lane_base + L::P_COL;
     float l = 0.0f, m_ref = -INFINITY;
     bool ok = true;
+    uint32_t mw = 0;
     for (int j = wg; j < nj; j += 2) {
       const int u = j >> 1;
-      const bool hi = is_hi(j);
+      if ((j & 31) == wg) mw = mrow[j >> 5];  // first tile of this group in a new mask word
+      const bool hi = (mw >> (j & 31)) & 1u;
       if (!__all_sync(0xffffffffu, mbar_wait(BAR(S_FULL + wg), u & 1, abort, kWaitLimitNs))) {
         raise_error(abort, 4u);
         ok = false;
         break;
       }
       tc_fence_after();
+      uint32_t v[128];
       const uint32_t s_addr = tmem + lane_base + L::S_COL0 + 128 * wg;
-      const bool edge = (p.causal && j == i) || ((j + 1) * 128 > p.N);  // warp-uniform
-      const int lim = min(p.causal ? row_g + 1 : p.N, p.N) - j * 128;    // columns >= lim are masked
-      // pass 1: row max of the raw logits (tree of three-input maxima)
+#pragma unroll
+      for (int c4 = 0; c4 < 4; ++c4) tmem_ld32(s_addr + 32 * c4, *reinterpret_cast<uint32_t(*)[32]>(&v[32 * c4]));
+      tmem_ld_wait();
+      // S is in registers: its TMEM buffer may take S_{j+2}
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(BAR(S_FREE + wg));
+      if ((p.causal && j == i) || ((j + 1) * 128 > p.N)) {  // warp-uniform: only edge tiles mask
+        const int lim = min(p.causal ? row_g + 1 : p.N, p.N) - j * 128;
+#pragma unroll
+        for (int c = 0; c < 128; ++c)
+          if (c >= lim) v[c] = __float_as_uint(-INFINITY);
+      }
+      // row max of the raw logits: a tree of three-input maxima
       float mloc;
       {
-        uint32_t v[128];
-#pragma unroll
-        for (int c4 = 0; c4 < 4; ++c4) tmem_ld32(s_addr + 32 * c4, *reinterpret_cast<uint32_t(*)[32]>(&v[32 * c4]));
-        tmem_ld_wait();
-        if (edge) {
-#pragma unroll
-          for (int c = 0; c < 128; ++c)
-            if (c >= lim) v[c] = __float_as_uint(-INFINITY);
-        }
         float t1[43];
 #pragma unroll
         for (int c = 0; c < 42; ++c)
@@ -317,33 +400,30 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float sc = hi ? sc_hi : sc_lo;
       float m_prev = -INFINITY;
       if (j > 0) {
-        named_bar_sync(bar_in, 64);
+        // m_{j-1} from the other group's warp of the same quarter
+        if (!__all_sync(0xffffffffu, mbar_wait(mx_in, ((j - 1) >> 1) & 1, abort, kWaitLimitNs))) {
+          raise_error(abort, 4u);
+          ok = false;
+          break;
+        }
         m_prev = mbuf[(wg ^ 1) * 128 + r];
       }
       const float m_new = fmaxf(m_prev, mloc * sc);
       mbuf[wg * 128 + r] = m_new;
-      if (j + 1 < nj) named_bar_arrive(bar_out, 64);
+      __syncwarp();
+      if (j + 1 < nj && lane == 0) mbar_arrive(mx_out);
       const float alpha = (m_prev == -INFINITY) ? 0.0f : ex2_approx(m_prev - m_new);  // O rescale
       const float beta = (m_ref == -INFINITY) ? 0.0f : ex2_approx(m_ref - m_new);     // own partial sum
       const uint64_t sc2 = f2pack(sc, sc);
       const uint64_t nb2 = f2pack(8.0f - m_new, 8.0f - m_new);  // p * 2^8 = 2^(s*sc - m_new + 8)
       uint64_t acc[4] = {0, 0, 0, 0};
-      // pass 2: exponentials by halves of 64 columns, re-read from TMEM
 #pragma unroll
-      for (int h2 = 0; h2 < 2; ++h2) {
-        uint32_t v[64];
-        tmem_ld32(s_addr + 64 * h2, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
-        tmem_ld32(s_addr + 64 * h2 + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
-        tmem_ld_wait();
-        if (edge) {
+      for (int ch = 0; ch < 4; ++ch) {  // chunks of 32 columns
+        uint32_t pw[16];
 #pragma unroll
-          for (int c = 0; c < 64; ++c)
-            if (64 * h2 + c >= lim) v[c] = __float_as_uint(-INFINITY);
-        }
-        uint32_t pw[32];
-#pragma unroll
-        for (int t = 0; t < 32; ++t) {  // element pairs
-          const uint64_t a2 = ffma2(f2pack(__uint_as_float(v[2 * t]), __uint_as_float(v[2 * t + 1])), sc2, nb2);
+        for (int t = 0; t < 16; ++t) {  // element pairs
+          const int c = 32 * ch + 2 * t;
+          const uint64_t a2 = ffma2(f2pack(__uint_as_float(v[c]), __uint_as_float(v[c + 1])), sc2, nb2);
           uint64_t e2;
           if ((t & 3) < NPOLY) {
             e2 = exp2_poly2(a2);
@@ -363,10 +443,21 @@ __global__ void __launch_bounds__(kThreads, 1)
             else pw[t >> 1] = hh;
           }
         }
-        // P overwrites the leading columns of this S buffer (those logits are already consumed)
-        if (hi) tmem_st32(s_addr + 32 * h2, pw);
-        else tmem_st16(s_addr + 16 * h2, *reinterpret_cast<uint32_t(*)[16]>(&pw[0]));
+        if (ch == 0 && !hi && j >= 3) {
+          // P region j % 3 was last read by an earlier FP4 tile's P.V, at the latest
+          // P_{j-3} V_{j-3}: wait until that product completed
+          if (!__all_sync(0xffffffffu, count_wait(pv_count, (uint32_t)(j - 2), abort, kWaitLimitNs))) {
+            raise_error(abort, 4u);
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+        }
+        // BF16 P overwrites the leading columns of this tile's own S buffer (already read)
+        if (hi) tmem_st16(s_addr + 16 * ch, pw);
+        else tmem_st8(p_base + 32 * (j % 3) + 8 * ch, *reinterpret_cast<uint32_t(*)[8]>(&pw[0]));
       }
+      if (!ok) break;
       float r0, r1, r2, r3, r4, r5, r6, r7;
       f2unpack(acc[0], r0, r1);
       f2unpack(acc[1], r2, r3);
@@ -375,9 +466,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       l = l * beta + (((r0 + r1) + (r2 + r3)) + ((r4 + r5) + (r6 + r7)));
       m_ref = m_new;
       // rescale O when any row of the warp has a new maximum (alpha == 1 is a no-op)
-      const bool corr = (j > 0) && (alpha != 1.0f);
-      if (__any_sync(0xffffffffu, corr)) {
-        if (!__all_sync(0xffffffffu, mbar_wait(BAR(PV_DONE), (j - 1) & 1, abort, kWaitLimitNs))) {
+      if (__any_sync(0xffffffffu, (j > 0) && (alpha != 1.0f))) {
+        if (!__all_sync(0xffffffffu, count_wait(pv_count, (uint32_t)j, abort, kWaitLimitNs))) {
           raise_error(abort, 4u);
           ok = false;
           break;
@@ -407,11 +497,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     // ---------------------------------------------------------- epilogue
     // combine the two groups' partial row sums, then each group writes D/2 columns
-    ok = ok && __all_sync(0xffffffffu, mbar_wait(BAR(O_FINAL), 0, abort, kWaitLimitNs));
-    float* xl = reinterpret_cast<float*>(smem + L::OFF_XCH) + 256;  // [2][128] sums, [2][128] maxima
+    ok = ok && __all_sync(0xffffffffu, count_wait(pv_count, (uint32_t)nj, abort, kWaitLimitNs));
+    float* xl = reinterpret_cast<float*>(smem + L::OFF_FIN);  // [2][128] sums, [2][128] maxima
     xl[wg * 128 + r] = l;
     xl[256 + wg * 128 + r] = m_ref;
-    named_bar_sync(9 + q4, 64);
+    named_bar_sync(1 + q4, 64);
     if (ok) {
       tc_fence_after();
       const float lo_ = xl[(wg ^ 1) * 128 + r], mo_ = xl[256 + (wg ^ 1) * 128 + r];
