@@ -32,7 +32,7 @@ if ROOT not in sys.path:
 
 import torch  # noqa: E402
 
-from mixed_precision_bit_quant_b200 import workloads  # noqa: E402
+from mixed_precision_bit_quant_b200 import dist as mdist, workloads  # noqa: E402
 
 METRIC = "attn TFLOPS (causal-adj) & % of mixed FP4/BF16 roofline, N=32K, 5% BF16"
 UNIT = "TFLOP/s"
@@ -46,13 +46,6 @@ def _peaks():
             d = json.load(f)
         return d, "measured"
     return dict(FALLBACK_PEAKS), "fallback"
-
-
-def _dist():
-    rank = int(os.environ.get("RANK", "0"))
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    return rank, world, local
 
 
 def hi_lo_pairs(w: workloads.Workload):
@@ -237,7 +230,7 @@ def cpu_baseline(w, q, k, v, n_tiles: int, seed: int = 1):
 
 
 def run_reference(args, w):
-    rank, world, _ = _dist()
+    rank, world, _ = mdist.env_ranks()
     if rank != 0:
         return 0
     q, k, v = workloads.generate(w)
@@ -295,18 +288,14 @@ def main():
 
     import mixed_precision_bit_quant_b200 as mq
 
-    rank, world, local = _dist()
+    rank, world, local = mdist.env_ranks()
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    pg = None
-    if world > 1:
-        import datetime
-        import torch.distributed as dist
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
-        pg = dist
+    mdist.init(dev)
     peaks, peak_src = _peaks()
 
-    q_h, k_h, v_h = workloads.generate(w)
+    # weak scaling: each rank owns an independent problem of the same shape (its own seed)
+    q_h, k_h, v_h = workloads.generate(mdist.rank_workload(w, rank))
     q, k, v = (t.to(dev) for t in (q_h, k_h, v_h))
     quant = mq.alloc_quantized(mq.shape_of(q, k, w.causal), dev)
     shape = mq.shape_of(q, k, w.causal)
@@ -346,8 +335,7 @@ def main():
     if sampler:
         sampler.start()
         time.sleep(0.6)  # nvidia-smi start-up
-    if pg:
-        pg.barrier()
+    mdist.barrier()
     torch.cuda.synchronize(dev)
     n0 = mq.launch_count()
     t_begin, t_end = ev(), ev()
@@ -360,8 +348,7 @@ def main():
     torch.cuda.synchronize(dev)
     if sampler:
         sampler.mark_stop()
-    if pg:
-        pg.barrier()
+    mdist.barrier()
     launches = mq.launch_count() - n0
     status, word = mq.device_status()
     if status != 0:
@@ -369,11 +356,7 @@ def main():
     if sampler:
         time.sleep(0.2)
         sampler.stop()
-    total_ms = t_begin.elapsed_time(t_end)
-    if pg:
-        tt = torch.tensor([total_ms], device=dev)
-        pg.all_reduce(tt, op=pg.ReduceOp.MAX)
-        total_ms = float(tt.item())
+    total_ms = mdist.max_over_ranks(t_begin.elapsed_time(t_end), dev)
     ms_step = total_ms / K
     q_ms = statistics.mean(m[0].elapsed_time(m[1]) for m in marks)
     s_ms = statistics.mean(m[1].elapsed_time(m[2]) for m in marks)
@@ -394,8 +377,7 @@ def main():
         for it in range(2 + ke):
             if it == 2:
                 torch.cuda.synchronize(dev)
-                if pg:
-                    pg.barrier()
+                mdist.barrier()
                 e0, e1 = ev(), ev()
                 e0.record(stream)
             q.copy_(qp, non_blocking=True)
@@ -405,11 +387,7 @@ def main():
             o_host.copy_(o, non_blocking=True)
         e1.record(stream)
         torch.cuda.synchronize(dev)
-        e_ms = e0.elapsed_time(e1) / ke
-        if pg:
-            tt = torch.tensor([e_ms], device=dev)
-            pg.all_reduce(tt, op=pg.ReduceOp.MAX)
-            e_ms = float(tt.item())
+        e_ms = mdist.max_over_ranks(e0.elapsed_time(e1) / ke, dev)
         h2d = sum(t.numel() * t.element_size() for t in (q_h, k_h, v_h))
         e2e = {"value": world * eff_flops / (e_ms * 1e-3) / 1e12, "unit": UNIT, "ms_per_step": e_ms,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": o_host.numel() * 2,
@@ -446,8 +424,7 @@ def main():
             "cpu_baseline": cpu,
         }
         print(json.dumps(line), flush=True)
-    if pg:
-        pg.destroy_process_group()
+    mdist.finalize()
     return 0
 
 

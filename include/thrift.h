@@ -190,6 +190,19 @@ THRIFT_API thrift_status thrift_attn_fwd(const thrift_shape *shape, const thrift
  */
 THRIFT_API thrift_status thrift_device_status(void *stream, uint32_t *detail);
 
+/*
+ * Test hook for the device watchdog.  After thrift_debug_withhold_v_load(t)
+ * with t >= 0, every later thrift_attn_fwd launch of this process skips the
+ * copy of key tile t's V operand in each work tile that reaches key tile t, so
+ * the product P_t V_t waits for data that never arrives.  That bounded wait
+ * gives up after 2 s; the work tile raises the abort flag, every role of it
+ * returns, its outputs are left undefined, and the next thrift_device_status
+ * reports THRIFT_ERR_TIMEOUT.  The CUDA context stays usable.  t < 0 turns the
+ * hook off (the default).  Process-wide; set it only while no launch is being
+ * issued from another thread.  Always returns THRIFT_OK.
+ */
+THRIFT_API thrift_status thrift_debug_withhold_v_load(int32_t tile);
+
 /* Human-readable name of a status code (static storage). */
 THRIFT_API const char *thrift_status_string(thrift_status status);
 

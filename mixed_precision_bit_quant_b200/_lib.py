@@ -69,6 +69,8 @@ def lib() -> ctypes.CDLL:
         L.thrift_device_status.restype = ctypes.c_int
         L.thrift_status_string.argtypes = [ctypes.c_int]
         L.thrift_status_string.restype = ctypes.c_char_p
+        L.thrift_debug_withhold_v_load.argtypes = [I32]
+        L.thrift_debug_withhold_v_load.restype = ctypes.c_int
         L.thrift_launch_count.argtypes = []
         L.thrift_launch_count.restype = U64
         L.thrift_version.argtypes = []
@@ -198,6 +200,11 @@ def device_status() -> tuple:
     w = ctypes.c_uint32(0)
     s = lib().thrift_device_status(_stream(), ctypes.byref(w))
     return int(s), int(w.value)
+
+
+def debug_withhold_v_load(tile: int) -> None:
+    """Watchdog test hook: later attention launches skip key tile `tile`'s V load (-1: off)."""
+    _check(lib().thrift_debug_withhold_v_load(int(tile)), "thrift_debug_withhold_v_load")
 
 
 def launch_count() -> int:

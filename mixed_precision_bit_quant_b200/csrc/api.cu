@@ -167,6 +167,11 @@ thrift_status thrift_device_status(void* stream, uint32_t* detail) {
   return w != 0 ? THRIFT_ERR_TIMEOUT : THRIFT_OK;
 }
 
+thrift_status thrift_debug_withhold_v_load(int32_t tile) {
+  set_withhold_v(tile);
+  return THRIFT_OK;
+}
+
 const char* thrift_status_string(thrift_status s) {
   switch (s) {
     case THRIFT_OK: return "THRIFT_OK";

@@ -30,12 +30,19 @@
 #include <cuda.h>
 #include <stdlib.h>
 
+#include <atomic>
+
 #include "dev.cuh"
 #include "kernels.h"
 
 namespace thrift {
 
 __device__ uint32_t g_attn_error_word;
+// Test hook for the device watchdog (thrift_debug_withhold_v_load): a key tile
+// whose V load the producer skips, so the P.V issuer's bounded wait runs out.
+static std::atomic<int> g_withhold_v{-1};
+
+void set_withhold_v(int tile) { g_withhold_v.store(tile < 0 ? -1 : tile, std::memory_order_relaxed); }
 
 namespace attn {
 
@@ -105,6 +112,7 @@ struct Params {
   float* lse;
   int B, Hq, Hkv, N, T, W, causal;
   float scale_log2;  // softmax scale * log2(e)
+  int withhold_v;    // test hook: key tile whose V load is never issued (-1: none)
 };
 
 __device__ __forceinline__ void raise_error(volatile int* abort, uint32_t code) {
@@ -161,6 +169,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto is_hi = [&](int j) -> bool { return (mrow[j >> 5] >> (j & 31)) & 1u; };
   volatile int never = 0;
   const uint32_t pv_count = sb + L::OFF_MISC + 8;  // number of completed P.V products, in tile order
+  int issued_lo = 0, issued_hi = 0;                 // loads a producer issued (drained on abort)
 
   if (warp >= 8) {
     regs_dec<kOtherRegs>();
@@ -201,7 +210,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             tma_load_3d(sb + L::OFF_KL + slot * L::KLO, &tm_kfp4, 0, j * 128, bhk, full);
             bulk_load(sb + L::OFF_KSF + slot * L::SF, p.k_sf_mma + ((size_t)bhk * p.T + j) * L::SF, L::SF, full);
           }
-        } else {
+        } else if (j != p.withhold_v) {
           if (hi) {
             const uint32_t vb = sb + L::OFF_VH + slot * L::VHI;
             mbar_expect_tx(full, L::VHI);
@@ -214,18 +223,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (hi) ++nhi; else ++nlo;
       }
-      if (*abort) {
-        // let copies already in flight land before the CTA's shared memory goes away
-        if (kside) mbar_wait(BAR(Q_FULL), 0, &never, kWaitLimitNs / 4);
-        for (int k = 0; k < NLO && k < nlo; ++k) {
-          const int n = nlo - 1 - k, slot = n % NLO;
-          mbar_wait(BAR((kside ? KL_FULL : VL_FULL) + slot), (n / NLO) & 1, &never, kWaitLimitNs / 4);
-        }
-        for (int k = 0; k < NHI && k < nhi; ++k) {
-          const int n = nhi - 1 - k, slot = n % NHI;
-          mbar_wait(BAR((kside ? KH_FULL : VH_FULL) + slot), (n / NHI) & 1, &never, kWaitLimitNs / 4);
-        }
-      }
+      issued_lo = nlo;
+      issued_hi = nhi;
     } else if (warp == 9 && lane == 0) {
       // ---------------------------------------------------------- QK^T issuer
       constexpr int KB = D / 64;
@@ -544,6 +543,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
+  if ((warp == 8 || warp == 10) && lane == 0 && *abort) {
+    // every role has returned and the abort flag is final: let the copies this
+    // producer issued land before the CTA's shared memory goes away (a copy that
+    // was never issued times out here after a quarter of the wait limit)
+    const bool kside = (warp == 8);
+    if (kside) mbar_wait(BAR(Q_FULL), 0, &never, kWaitLimitNs / 4);
+    for (int k = 0; k < NLO && k < issued_lo; ++k) {
+      const int n = issued_lo - 1 - k, slot = n % NLO;
+      mbar_wait(BAR((kside ? KL_FULL : VL_FULL) + slot), (n / NLO) & 1, &never, kWaitLimitNs / 4);
+    }
+    for (int k = 0; k < NHI && k < issued_hi; ++k) {
+      const int n = issued_hi - 1 - k, slot = n % NHI;
+      mbar_wait(BAR((kside ? KH_FULL : VH_FULL) + slot), (n / NHI) & 1, &never, kWaitLimitNs / 4);
+    }
+  }
 }
 
 // ---------------------------------------------------------------------------
@@ -624,6 +638,7 @@ static int launch_d(const AttnArgs& a, cudaStream_t st) {
   p.B = a.B; p.Hq = a.Hq; p.Hkv = a.Hkv; p.N = a.N; p.T = T; p.W = W; p.causal = a.causal;
   const float scale = a.softmax_scale > 0.0f ? a.softmax_scale : 1.0f / sqrtf((float)D);
   p.scale_log2 = scale * 1.4426950408889634f;
+  p.withhold_v = g_withhold_v.load(std::memory_order_relaxed);
   auto kern = attn_fwd_kernel<D, 0>;
   switch (exp_poly_pairs()) {
     case 1: kern = attn_fwd_kernel<D, 1>; break;

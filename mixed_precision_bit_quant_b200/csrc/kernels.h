@@ -44,5 +44,6 @@ struct AttnArgs {
 int launch_attn(const AttnArgs& a, cudaStream_t s);
 
 cudaError_t read_and_clear_device_error(cudaStream_t s, uint32_t* word);
+void set_withhold_v(int tile);  // watchdog test hook (-1: off)
 
 }  // namespace thrift
