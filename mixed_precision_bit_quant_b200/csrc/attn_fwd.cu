@@ -60,7 +60,13 @@ enum Bar : int {
   Q_FULL = 0,
   KL_FULL = 1, KL_EMPTY = KL_FULL + NLO, VL_FULL = KL_EMPTY + NLO, VL_EMPTY = VL_FULL + NLO,
   KH_FULL = VL_EMPTY + NLO, KH_EMPTY = KH_FULL + NHI, VH_FULL = KH_EMPTY + NHI, VH_EMPTY = VH_FULL + NHI,
-  S_FULL = VH_EMPTY + NHI, S_FREE = S_FULL + 2, P_FULL = S_FREE + 2, PVC = P_FULL + 2,
+  // P_FULL is a ring of four barriers per softmax group, indexed by the group's
+  // tile count u: a group can finish a tile before the P.V issuer has waited on
+  // the group's previous one (a BF16 tile needs no P region), so one barrier per
+  // group could complete two phases under the issuer.  Before the group finishes
+  // its tile u+3, either its FP4 tile waited for P.V up to a tile after u or a
+  // BF16 predecessor's S buffer waited for that tile's P.V, so four slots never alias.
+  S_FULL = VH_EMPTY + NHI, S_FREE = S_FULL + 2, P_FULL = S_FREE + 2, PVC = P_FULL + 8,
   QK_DRAIN = PVC + 2, PV_DRAIN = QK_DRAIN + 1,
   MX = PV_DRAIN + 1,  // running-max hand-off [group][quarter]
   NBAR = MX + 8
@@ -149,7 +155,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (tid == 0) {
     for (int k = 0; k < NBAR; ++k) {
-      const bool by_group = (k >= S_FREE && k < S_FREE + 2) || (k >= P_FULL && k < P_FULL + 2);
+      const bool by_group = (k >= S_FREE && k < S_FREE + 2) || (k >= P_FULL && k < P_FULL + 8);
       mbar_init(BAR(k), by_group ? 4 : 1);  // softmax barriers: one arrival per warp of the group
     }
     *abort = 0;
@@ -297,7 +303,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const bool hi = (mw >> (t & 31)) & 1u;
         const int s = t & 1, u = t >> 1;
         const int n = hi ? n_hi : n_lo, slots = hi ? NHI : NLO, slot = n % slots, use = n / slots;
-        if (!mbar_wait(BAR(P_FULL + s), u & 1, abort, kWaitLimitNs) ||
+        if (!mbar_wait(BAR(P_FULL + 4 * s + (u & 3)), (u >> 2) & 1, abort, kWaitLimitNs) ||
             !mbar_wait(BAR((hi ? VH_FULL : VL_FULL) + slot), use & 1, abort, kWaitLimitNs)) {
           ok = false;
           break;
@@ -492,7 +498,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(BAR(P_FULL + wg));
+      if (lane == 0) mbar_arrive(BAR(P_FULL + 4 * wg + (u & 3)));
     }
     // ---------------------------------------------------------- epilogue
     // combine the two groups' partial row sums, then each group writes D/2 columns

@@ -123,11 +123,14 @@ __device__ __forceinline__ uint32_t ld_acquire_u32(uint32_t addr) {
   asm volatile("ld.acquire.cta.shared::cta.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
   return v;
 }
-// Bounded wait until the counter at `addr` reaches `target`.
+// Bounded wait until the counter at `addr` reaches `target`.  Between polls the
+// thread sleeps briefly, so a waiting warp leaves its issue slots to the warps
+// that compute.
 __device__ __forceinline__ bool count_wait(uint32_t addr, uint32_t target, volatile int* abort, uint64_t limit_ns) {
   if (ld_acquire_u32(addr) >= target) return true;
   uint64_t t0 = globaltimer_ns();
   for (uint32_t it = 1;; ++it) {
+    __nanosleep(20);
     if (ld_acquire_u32(addr) >= target) return true;
     if ((it & 63u) == 0u) {
       if (*abort) return false;
