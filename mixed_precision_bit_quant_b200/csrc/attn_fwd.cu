@@ -21,10 +21,14 @@
 //              S = Q4 K4^T kind::mxf4nvf4 (block scales in TMEM), BF16 pair
 //              S = Q K^T kind::f16; S of tile j+2 as soon as group j%2 read S_j.
 //   warp 11    P.V issuer (one thread): O += P8 V8 kind::f8f6f4 or O += P16 Vs
-//              kind::f16, P read from TMEM; publishes the count of completed
-//              products in shared memory (the only P.V progress signal).
+//              kind::f16, P read from TMEM; each product's completion is committed
+//              to a ring of mbarriers that the softmax groups wait on before
+//              they reuse a P region or rescale O.
 //   Warps 8-11 form the third warpgroup, whose registers the softmax warps
 //   take over with setmaxnreg.
+// The exponentials of a 32-column chunk form one branch-free block that makes
+// both P encodings (e4m3 and bf16); one copy of this block serves FP4 and BF16
+// tiles alike, which keeps the loop small enough for the instruction cache.
 // TMEM columns: S double buffer [0,256), O [256,256+D), three 32-column e4m3 P
 // regions [256+D, 352+D) (BF16 tiles keep P in their S buffer), block scales after.
 #include <cuda.h>
@@ -50,7 +54,6 @@ constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s per wait: far above any
 constexpr int kThreads = 384;                       // 8 softmax warps + 4 producer / issuer warps
 constexpr int kSoftmaxRegs = 224, kOtherRegs = 56;  // 256*224 + 128*56 = 384*168 (the launch budget)
 constexpr int kMaxW = 128;                          // mask words per query tile (T <= 4096)
-constexpr int kDefaultPolyPairs = 0;
 
 // Operand rings: FP4 tiles use NLO slots of K (e2m1 + scales) and of V^T (e4m3);
 // BF16 tiles use NHI slots of bf16 K and V^T.  Producer and MMA issuer walk the
@@ -66,8 +69,9 @@ enum Bar : int {
   // group could complete two phases under the issuer.  Before the group finishes
   // its tile u+3, either its FP4 tile waited for P.V up to a tile after u or a
   // BF16 predecessor's S buffer waited for that tile's P.V, so four slots never alias.
+  // PVC is the ring of P.V completion barriers (see pv_wait).
   S_FULL = VH_EMPTY + NHI, S_FREE = S_FULL + 2, P_FULL = S_FREE + 2, PVC = P_FULL + 8,
-  QK_DRAIN = PVC + 2, PV_DRAIN = QK_DRAIN + 1,
+  QK_DRAIN = PVC + 8, PV_DRAIN = QK_DRAIN + 1,
   MX = PV_DRAIN + 1,  // running-max hand-off [group][quarter]
   NBAR = MX + 8
 };
@@ -126,7 +130,7 @@ __device__ __forceinline__ void raise_error(volatile int* abort, uint32_t code) 
   atomicOr(&g_attn_error_word, code);
 }
 
-template <int D, int NPOLY>
+template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_qfp4, const __grid_constant__ CUtensorMap tm_kfp4,
                     const __grid_constant__ CUtensorMap tm_qbf, const __grid_constant__ CUtensorMap tm_kbf,
@@ -174,7 +178,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = *tmem_holder;
   auto is_hi = [&](int j) -> bool { return (mrow[j >> 5] >> (j & 31)) & 1u; };
   volatile int never = 0;
-  const uint32_t pv_count = sb + L::OFF_MISC + 8;  // number of completed P.V products, in tile order
+  // P_t V_t completion: tcgen05.commit to PVC[t % 8] (products complete in issue order).  A
+  // waiter for tile t cannot see the barrier two phases ahead: P_{t+8} comes from the group
+  // of tile t, which needs m_{t+7} from the other group, i.e. every wait for P_t V_t came first.
+  auto pv_wait = [&](int t) -> bool { return mbar_wait(BAR(PVC + (t & 7)), (t >> 3) & 1, abort, kWaitLimitNs); };
   int issued_lo = 0, issued_hi = 0;                 // loads a producer issued (drained on abort)
 
   if (warp >= 8) {
@@ -254,7 +261,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (j >= 2) {
           if (!mbar_wait(BAR(S_FREE + s), ((j - 2) >> 1) & 1, abort, kWaitLimitNs)) { ok = false; break; }
           if (((j - 2) >> 5) == (j >> 5) ? ((mw >> ((j - 2) & 31)) & 1u) : is_hi(j - 2)) {
-            if (!count_wait(pv_count, (uint32_t)(j - 1), abort, kWaitLimitNs)) { ok = false; break; }
+            if (!pv_wait(j - 2)) { ok = false; break; }
           }
         }
         const int n = hi ? n_hi : n_lo, slots = hi ? NHI : NLO, slot = n % slots, use = n / slots;
@@ -329,10 +336,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_commit(BAR(VL_EMPTY + slot));
           ++n_lo;
         }
-        tc_commit(BAR(PVC + s));
-        if (!mbar_wait(BAR(PVC + s), u & 1, abort, kWaitLimitNs)) { ok = false; break; }
-        tc_fence_after();
-        st_release_u32(pv_count, (uint32_t)(t + 1));
+        tc_commit(BAR(PVC + (t & 7)));
       }
       if (!ok) raise_error(abort, 2u);
       tc_commit(BAR(PV_DRAIN));
@@ -422,45 +426,45 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t sc2 = f2pack(sc, sc);
       const uint64_t nb2 = f2pack(8.0f - m_new, 8.0f - m_new);  // p * 2^8 = 2^(s*sc - m_new + 8)
       uint64_t acc[4] = {0, 0, 0, 0};
+      uint32_t pe_all[32];
 #pragma unroll
       for (int ch = 0; ch < 4; ++ch) {  // chunks of 32 columns
-        uint32_t pw[16];
+        // both P encodings for every pair (no branch in the loop: one basic block per
+        // chunk whose pairs overlap); the store below takes the one the tile needs
+        uint32_t pb[16], pe[8];
 #pragma unroll
         for (int t = 0; t < 16; ++t) {  // element pairs
           const int c = 32 * ch + 2 * t;
           const uint64_t a2 = ffma2(f2pack(__uint_as_float(v[c]), __uint_as_float(v[c + 1])), sc2, nb2);
-          uint64_t e2;
-          if ((t & 3) < NPOLY) {
-            e2 = exp2_poly2(a2);
-          } else {
-            float a0, a1;
-            f2unpack(a2, a0, a1);
-            e2 = f2pack(ex2_approx(a0), ex2_approx(a1));
-          }
+          float a0, a1;
+          f2unpack(a2, a0, a1);
+          const uint64_t e2 = f2pack(ex2_approx(a0), ex2_approx(a1));
           acc[t & 3] = fadd2(acc[t & 3], e2);
           float e0, e1;
           f2unpack(e2, e0, e1);
-          if (hi) {
-            pw[t] = cvt_bf16x2(e0, e1);
-          } else {
-            const uint32_t hh = cvt_e4m3x2(e0, e1);
-            if (t & 1) pw[t >> 1] = __byte_perm(pw[t >> 1], hh, 0x5410);
-            else pw[t >> 1] = hh;
-          }
+          pb[t] = cvt_bf16x2(e0, e1);
+          const uint32_t hh = cvt_e4m3x2(e0, e1);
+          if (t & 1) pe[t >> 1] = __byte_perm(pe[t >> 1], hh, 0x5410);
+          else pe[t >> 1] = hh;
         }
-        if (ch == 0 && !hi && j >= 3) {
+        // BF16 P overwrites the leading columns of this tile's own S buffer (already read);
+        // the e4m3 P of an FP4 tile is stored once, after its P region is free
+        if (hi) tmem_st16(s_addr + 16 * ch, pb);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) pe_all[8 * ch + q] = pe[q];
+      }
+      if (!hi) {
+        if (j >= 3) {
           // P region j % 3 was last read by an earlier FP4 tile's P.V, at the latest
-          // P_{j-3} V_{j-3}: wait until that product completed
-          if (!__all_sync(0xffffffffu, count_wait(pv_count, (uint32_t)(j - 2), abort, kWaitLimitNs))) {
+          // P_{j-3} V_{j-3}: wait (after the exponentials) until that product completed
+          if (!__all_sync(0xffffffffu, pv_wait(j - 3))) {
             raise_error(abort, 4u);
             ok = false;
-            break;
+          } else {
+            tc_fence_after();
           }
-          tc_fence_after();
         }
-        // BF16 P overwrites the leading columns of this tile's own S buffer (already read)
-        if (hi) tmem_st16(s_addr + 16 * ch, pw);
-        else tmem_st8(p_base + 32 * (j % 3) + 8 * ch, *reinterpret_cast<uint32_t(*)[8]>(&pw[0]));
+        if (ok) tmem_st32(p_base + 32 * (j % 3), pe_all);
       }
       if (!ok) break;
       float r0, r1, r2, r3, r4, r5, r6, r7;
@@ -472,7 +476,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       m_ref = m_new;
       // rescale O when any row of the warp has a new maximum (alpha == 1 is a no-op)
       if (__any_sync(0xffffffffu, (j > 0) && (alpha != 1.0f))) {
-        if (!__all_sync(0xffffffffu, count_wait(pv_count, (uint32_t)j, abort, kWaitLimitNs))) {
+        if (!__all_sync(0xffffffffu, pv_wait(j - 1))) {
           raise_error(abort, 4u);
           ok = false;
           break;
@@ -502,7 +506,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     // ---------------------------------------------------------- epilogue
     // combine the two groups' partial row sums, then each group writes D/2 columns
-    ok = ok && __all_sync(0xffffffffu, count_wait(pv_count, (uint32_t)nj, abort, kWaitLimitNs));
+    ok = ok && __all_sync(0xffffffffu, pv_wait(nj - 1));
     float* xl = reinterpret_cast<float*>(smem + L::OFF_FIN);  // [2][128] sums, [2][128] maxima
     xl[wg * 128 + r] = l;
     xl[256 + wg * 128 + r] = m_ref;
@@ -599,18 +603,6 @@ static bool make_map(CUtensorMap* m, CUtensorMapDataType dt, const void* base, u
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Share of exponentials computed by the FMA-pipe polynomial instead of the MUFU
-// unit: npoly of every 4 element pairs.  Tunable with THRIFT_EXP_POLY (0..2).
-static int exp_poly_pairs() {
-  static int v = -1;
-  if (v < 0) {
-    const char* e = getenv("THRIFT_EXP_POLY");
-    int x = e ? atoi(e) : kDefaultPolyPairs;
-    v = x < 0 ? 0 : (x > 2 ? 2 : x);
-  }
-  return v;
-}
-
 template <int D>
 static int launch_d(const AttnArgs& a, cudaStream_t st) {
   using L = Layout<D>;
@@ -645,12 +637,7 @@ static int launch_d(const AttnArgs& a, cudaStream_t st) {
   const float scale = a.softmax_scale > 0.0f ? a.softmax_scale : 1.0f / sqrtf((float)D);
   p.scale_log2 = scale * 1.4426950408889634f;
   p.withhold_v = g_withhold_v.load(std::memory_order_relaxed);
-  auto kern = attn_fwd_kernel<D, 0>;
-  switch (exp_poly_pairs()) {
-    case 1: kern = attn_fwd_kernel<D, 1>; break;
-    case 2: kern = attn_fwd_kernel<D, 2>; break;
-    default: break;
-  }
+  auto kern = attn_fwd_kernel<D>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::DYN) != cudaSuccess)
     return THRIFT_ERR_CUDA;
   const unsigned grid = (unsigned)(BHq * (uint64_t)T);

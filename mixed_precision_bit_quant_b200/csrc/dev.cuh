@@ -356,37 +356,6 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   return d;
 }
 
-// 2^x for two arguments on the FMA pipe (x <= 128).  x is clamped to >= -127;
-// n = floor(x) by adding 1.5 * 2^23 with round-toward-minus-infinity, f = x - n in
-// [0, 1) exactly, 2^f by a degree-4 polynomial (coefficients fitted here by
-// relative-error least squares on [0, 1): max relative error 2.7e-6 in FP32),
-// and n is added to the exponent field of the result.
-__device__ __forceinline__ uint64_t exp2_poly2(uint64_t x2) {
-  float x0, x1;
-  f2unpack(x2, x0, x1);
-  x0 = fmaxf(x0, -127.0f);
-  x1 = fmaxf(x1, -127.0f);
-  x2 = f2pack(x0, x1);
-  const uint64_t C = f2pack(12582912.0f, 12582912.0f);
-  const uint64_t t2 = fadd2_rm(x2, C);                       // 1.5*2^23 + floor(x)
-  const uint64_t nC = f2pack(-12582912.0f, -12582912.0f);
-  const uint64_t n2 = fadd2(t2, nC);                          // floor(x), exact
-  float n0, n1;
-  f2unpack(n2, n0, n1);
-  const uint64_t f2 = fadd2(x2, f2pack(-n0, -n1));            // x - floor(x), exact
-  uint64_t p = f2pack(1.3534157536923885e-2f, 1.3534157536923885e-2f);
-  p = ffma2(p, f2, f2pack(5.2011482417583466e-2f, 5.2011482417583466e-2f));
-  p = ffma2(p, f2, f2pack(2.414427399635315e-1f, 2.414427399635315e-1f));
-  p = ffma2(p, f2, f2pack(6.930038332939148e-1f, 6.930038332939148e-1f));
-  p = ffma2(p, f2, f2pack(1.0000026226043701f, 1.0000026226043701f));
-  float p0, p1, t0, t1;
-  f2unpack(p, p0, p1);
-  f2unpack(t2, t0, t1);
-  const float r0 = __uint_as_float(__float_as_uint(p0) + (__float_as_uint(t0) << 23));
-  const float r1 = __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23));
-  return f2pack(r0, r1);
-}
-
 // ---------------------------------------------------------------------------
 // Conversions for P.
 // ---------------------------------------------------------------------------

@@ -59,116 +59,152 @@ __device__ __forceinline__ uint32_t order_key(float f) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-template <int NT>
-__device__ __forceinline__ int block_sum(int v, int* red) {
-  v = __reduce_add_sync(0xffffffffu, v);
-  const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
-  __syncthreads();
-  if (l == 0) red[w] = v;
-  __syncthreads();
-  int s = 0;
-#pragma unroll
-  for (int i = 0; i < NT / 32; ++i) s += red[i];
-  return s;
-}
-
-// Scores + selection for one (b, hq, query tile i).  grid (T, B*Hq), 256 threads.
-// Dynamic shared memory: T keys (uint32) + T selection bytes.
-template <int D>
-__global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ qp, const float* __restrict__ kpT,
-                                                   int Hq, int Hkv, int T, int W, int causal, int budget_bp,
-                                                   int budget_tiles, uint32_t* __restrict__ mask,
-                                                   int32_t* __restrict__ counts) {
-  constexpr int NT = 256;
-  extern __shared__ uint32_t dyn[];
-  uint32_t* key = dyn;
-  uint8_t* sel = reinterpret_cast<uint8_t*>(dyn + T);
-  __shared__ float qs[D];
-  __shared__ int red[NT / 32];
-  __shared__ int eq_base;
-  const int i = blockIdx.x, bhq = blockIdx.y;
+// Scores + selection for R consecutive query tiles of one (b, hq).
+// grid (ceil(T / R), B*Hq), 32*R threads: R warps.
+// Scores: thread t takes the key tiles j = t, t + 32R, ... and accumulates the R
+// rows' dot products together, so each pooled key column is read once per CTA.
+// Selection: warp r takes query tile i0 + r and finds the kprime-th largest
+// candidate key by a 4-pass radix select (8-bit digits, per-warp histogram in
+// shared memory); keys above it are taken, keys equal to it in ascending tile
+// order until the budget is met.  Dynamic shared memory: R * T keys (uint32).
+template <int D, int R>
+__global__ void __launch_bounds__(32 * R) topk_kernel(const float* __restrict__ qp, const float* __restrict__ kpT,
+                                                      int Hq, int Hkv, int T, int W, int causal, int budget_bp,
+                                                      int budget_tiles, uint32_t* __restrict__ mask,
+                                                      int32_t* __restrict__ counts) {
+  constexpr int NT = 32 * R;
+  extern __shared__ uint32_t keys[];  // [R][T]
+  __shared__ float qs[R][D];
+  __shared__ uint32_t hist[R][256];
+  const int i0 = blockIdx.x * R, bhq = blockIdx.y;
   const int b = bhq / Hq, h = bhq % Hq;
   const int bhk = b * Hkv + h / (Hq / Hkv);
-  for (int c = threadIdx.x; c < D; c += NT) qs[c] = qp[((long long)bhq * T + i) * D + c];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  for (int x = threadIdx.x; x < R * D; x += NT) {
+    const int r = x / D, c = x % D;
+    qs[r][c] = (i0 + r < T) ? qp[((long long)bhq * T + i0 + r) * D + c] : 0.0f;
+  }
   __syncthreads();
 
-  const int n_i = causal ? i + 1 : T;
-  const int nf = (i == 0) ? 1 : 2;  // forced {0, i}, both always candidates
-  int k_i;
-  if (budget_tiles > 0) k_i = min(n_i, max(nf, budget_tiles));
-  else if (budget_bp <= 0) k_i = 0;
-  else if (budget_bp >= 10000) k_i = n_i;
-  else k_i = min(n_i, max(nf, (int)(((long long)budget_bp * n_i + 9999) / 10000)));
-  const int kprime = k_i > 0 ? k_i - nf : 0;
+  // per-row budget: forced {0, i} count toward k_i
+  auto budget = [&](int i, int& n_i, int& nf, int& k_i) {
+    n_i = causal ? i + 1 : T;
+    nf = (i == 0) ? 1 : 2;
+    if (budget_tiles > 0) k_i = min(n_i, max(nf, budget_tiles));
+    else if (budget_bp <= 0) k_i = 0;
+    else if (budget_bp >= 10000) k_i = n_i;
+    else k_i = min(n_i, max(nf, (int)(((long long)budget_bp * n_i + 9999) / 10000)));
+  };
 
+  // scores in FP32, channels in ascending order, separately rounded multiply and add
   const float* kcol = kpT + (long long)bhk * D * T;
-  for (int j = threadIdx.x; j < T; j += NT) {
-    uint32_t kk = 0;
-    const bool forced = (j == 0 || j == i);
-    if (j < n_i && !forced && kprime > 0) {
-      float acc = 0.0f;
-#pragma unroll 8
-      for (int c = 0; c < D; ++c) acc = __fadd_rn(acc, __fmul_rn(qs[c], __ldg(kcol + (long long)c * T + j)));
-      kk = order_key(acc);
+  const int jmax = causal ? min(T, i0 + R) : T;  // no row of this CTA looks past it
+  for (int j = threadIdx.x; j < jmax; j += NT) {
+    float acc[R];
+#pragma unroll
+    for (int r = 0; r < R; ++r) acc[r] = 0.0f;
+#pragma unroll 16
+    for (int c = 0; c < D; ++c) {
+      const float kv = __ldg(kcol + (long long)c * T + j);
+#pragma unroll
+      for (int r = 0; r < R; ++r) acc[r] = __fadd_rn(acc[r], __fmul_rn(qs[r][c], kv));
     }
-    key[j] = kk;
-    sel[j] = (k_i > 0 && forced && j < n_i) ? 1 : 0;
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      const int i = i0 + r;
+      uint32_t kk = 0;  // 0: not a candidate
+      if (i < T) {
+        int n_i, nf, k_i;
+        budget(i, n_i, nf, k_i);
+        if (j < n_i && j != 0 && j != i && k_i > nf) kk = order_key(acc[r]);
+      }
+      keys[r * T + j] = kk;
+    }
   }
   __syncthreads();
 
+  const int i = i0 + warp;
+  if (i >= T) return;
+  int n_i, nf, k_i;
+  budget(i, n_i, nf, k_i);
+  const int kprime = k_i > 0 ? k_i - nf : 0;
+  const uint32_t* key = keys + warp * T;
+  const int jend = causal ? n_i : T;
+  uint32_t tau = 0xFFFFFFFFu;  // no candidate key reaches it when kprime == 0
+  int need_eq = 0;
   if (kprime > 0) {
-    // tau = the kprime-th largest key among candidates (bitwise search).
-    uint32_t tau = 0;
-    for (int bit = 31; bit >= 0; --bit) {
-      const uint32_t cand = tau | (1u << bit);
-      int cnt = 0;
-      for (int j = threadIdx.x; j < T; j += NT) cnt += (key[j] >= cand) ? 1 : 0;
-      if (block_sum<NT>(cnt, red) >= kprime) tau = cand;
-    }
-    int gt = 0;
-    for (int j = threadIdx.x; j < T; j += NT) gt += (key[j] > tau) ? 1 : 0;
-    const int n_gt = block_sum<NT>(gt, red);
-    const int need_eq = kprime - n_gt;  // >= 1
-    if (threadIdx.x == 0) eq_base = 0;
-    __syncthreads();
-    // keys > tau all selected; keys == tau selected in ascending index order.
-    for (int j0 = 0; j0 < T; j0 += NT) {
-      const int j = j0 + threadIdx.x;
-      const bool eq = (j < T) && key[j] == tau;
-      const uint32_t bal = __ballot_sync(0xffffffffu, eq);
-      const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-      __syncthreads();
-      if (lane == 0) red[w] = __popc(bal);
-      __syncthreads();
-      int before = eq_base;
-      for (int q = 0; q < w; ++q) before += red[q];
-      before += __popc(bal & ((1u << lane) - 1u));
-      if (j < T) {
-        if (key[j] > tau) sel[j] = 1;
-        else if (eq && before < need_eq) sel[j] = 1;
+    uint32_t prefix = 0, pmask = 0;
+    int remaining = kprime;  // keys still to take among those matching the prefix
+#pragma unroll 1
+    for (int pass = 0; pass < 4; ++pass) {
+      const int shift = 24 - 8 * pass;
+#pragma unroll
+      for (int q = 0; q < 8; ++q) hist[warp][lane * 8 + q] = 0u;
+      __syncwarp();
+      for (int j = lane; j < jend; j += 32) {
+        const uint32_t k = key[j];
+        if (k != 0u && (k & pmask) == prefix) atomicAdd(&hist[warp][(k >> shift) & 255u], 1u);
       }
-      __syncthreads();
-      if (threadIdx.x == 0) {
-        int s = 0;
-        for (int q = 0; q < NT / 32; ++q) s += red[q];
-        eq_base += s;
+      __syncwarp();
+      // lane l owns digits [8l, 8l+8); counts above each lane's range by a suffix scan
+      uint32_t hv[8];
+      uint32_t lsum = 0;
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        hv[q] = hist[warp][lane * 8 + q];
+        lsum += hv[q];
       }
-      __syncthreads();
+      uint32_t above = lsum;  // inclusive suffix sum over lanes >= this one
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t t = __shfl_down_sync(0xffffffffu, above, o);
+        if (lane + o < 32) above += t;
+      }
+      const uint32_t above_excl = above - lsum;  // keys in higher lanes' digits
+      // the lane whose range holds the remaining-th largest key
+      const bool mine = above_excl < (uint32_t)remaining && above >= (uint32_t)remaining;
+      int digit = 0, rem_new = 0;
+      if (mine) {
+        uint32_t cum = above_excl;
+#pragma unroll
+        for (int q = 7; q >= 0; --q) {
+          if (cum + hv[q] >= (uint32_t)remaining) {
+            digit = lane * 8 + q;
+            rem_new = remaining - (int)cum;
+            break;
+          }
+          cum += hv[q];
+        }
+      }
+      const uint32_t bal = __ballot_sync(0xffffffffu, mine);
+      const int src = __ffs(bal) - 1;
+      digit = __shfl_sync(0xffffffffu, digit, src);
+      rem_new = __shfl_sync(0xffffffffu, rem_new, src);
+      prefix |= (uint32_t)digit << shift;
+      pmask |= 0xFFu << shift;
+      remaining = rem_new;
+      __syncwarp();
     }
+    tau = prefix;           // the kprime-th largest candidate key
+    need_eq = remaining;    // how many keys equal to tau are taken (>= 1)
   }
-  __syncthreads();
-  // pack the bitmask: one warp per 32-tile word
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  int pc = 0;
-  for (int wd = warp; wd < W; wd += NT / 32) {
+  // bit j set: forced tile, key above tau, or one of the first need_eq keys equal to tau
+  int eq_seen = 0, total = 0;
+  for (int wd = 0; wd < W; ++wd) {
     const int j = wd * 32 + lane;
-    const bool bit = (j < T) && sel[j];
+    const uint32_t k = (j < jend) ? key[j] : 0u;  // keys past the causal limit were never written
+    const bool eq = k != 0u && k == tau;
+    const uint32_t beq = __ballot_sync(0xffffffffu, eq);
+    const int before = eq_seen + __popc(beq & ((1u << lane) - 1u));
+    const bool forced = k_i > 0 && j < n_i && (j == 0 || j == i);
+    const bool bit = forced || (k != 0u && k > tau && kprime > 0) || (eq && before < need_eq);
     const uint32_t word = __ballot_sync(0xffffffffu, bit);
     if (lane == 0) mask[((long long)bhq * T + i) * W + wd] = word;
-    pc += (lane == 0) ? __popc(word) : 0;
+    eq_seen += __popc(beq);
+    total += __popc(word);
   }
-  const int total = block_sum<NT>(pc, red);
-  if (counts != nullptr && threadIdx.x == 0) counts[(long long)bhq * T + i] = total;
+  if (counts != nullptr && lane == 0) counts[(long long)bhq * T + i] = total;
 }
 
 cudaError_t launch_select(const SelectArgs& a, cudaStream_t s) {
@@ -177,17 +213,19 @@ cudaError_t launch_select(const SelectArgs& a, cudaStream_t s) {
   float* qp = a.pool_ws;
   float* kpT = qp + (size_t)BHq * T * D;
   dim3 gp(T, BHq + BHk);
-  const size_t dyn = (size_t)T * 5 + 16;
+  constexpr int R = 8;
+  const size_t dyn = (size_t)R * T * 4;
+  const dim3 gt((T + R - 1) / R, BHq);
   if (D == 128) {
     pool_kernel<128><<<gp, 64, 0, s>>>(a.q, a.k, BHq, a.N, T, qp, kpT);
-    if (dyn > 48 * 1024) cudaFuncSetAttribute(topk_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dyn);
-    topk_kernel<128><<<dim3(T, BHq), 256, dyn, s>>>(qp, kpT, a.Hq, a.Hkv, T, W, a.causal, a.budget_bp,
-                                                    a.budget_tiles, a.mask, a.counts);
+    if (dyn > 48 * 1024) cudaFuncSetAttribute(topk_kernel<128, R>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dyn);
+    topk_kernel<128, R><<<gt, 32 * R, dyn, s>>>(qp, kpT, a.Hq, a.Hkv, T, W, a.causal, a.budget_bp, a.budget_tiles,
+                                                a.mask, a.counts);
   } else {
     pool_kernel<64><<<gp, 32, 0, s>>>(a.q, a.k, BHq, a.N, T, qp, kpT);
-    if (dyn > 48 * 1024) cudaFuncSetAttribute(topk_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dyn);
-    topk_kernel<64><<<dim3(T, BHq), 256, dyn, s>>>(qp, kpT, a.Hq, a.Hkv, T, W, a.causal, a.budget_bp,
-                                                   a.budget_tiles, a.mask, a.counts);
+    if (dyn > 48 * 1024) cudaFuncSetAttribute(topk_kernel<64, R>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dyn);
+    topk_kernel<64, R><<<gt, 32 * R, dyn, s>>>(qp, kpT, a.Hq, a.Hkv, T, W, a.causal, a.budget_bp, a.budget_tiles,
+                                               a.mask, a.counts);
   }
   count_launches(2);
   return cudaGetLastError();
