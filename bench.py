@@ -81,8 +81,9 @@ def attn_roofline(w: workloads.Workload, peaks: dict, key: str = "bf16_tflops"):
     p16 = peaks[key] * 1e12
     p8, p4 = 2 * p16, 4 * p16
     t = lo * (F / p4 + F / p8) + hi * (2 * F / p16)
+    t_fp4_both = lo * (2 * F / p4) + hi * (2 * F / p16)  # stricter: P V at the FP4 rate too
     flops = (hi + lo) * 2 * F
-    return dict(flops=flops, t_roof=t, peak=flops / t, hi=hi, lo=lo)
+    return dict(flops=flops, t_roof=t, peak=flops / t, hi=hi, lo=lo, t_roof_fp4_both=t_fp4_both)
 
 
 def attn_algorithmic_bytes(w: workloads.Workload, hi: int, lo: int) -> float:
@@ -411,7 +412,8 @@ def main():
                          "unit": "TFLOP/s", "frac": achieved / peak, "traffic": traffic,
                          "peak_source": f"{peak_src} bf16 {peaks['bf16_tflops']} TF/s burst; FP8 = 2x, FP4 = 4x "
                                         f"(nominal dense ratios); BF16 pairs {roof['hi']}, FP4 pairs {roof['lo']}",
-                         "t_roof_ms": roof["t_roof"] * 1e3, "algorithmic_flops": roof["flops"]},
+                         "t_roof_ms": roof["t_roof"] * 1e3, "algorithmic_flops": roof["flops"],
+                         "frac_if_pv_at_fp4_rate": roof["t_roof_fp4_both"] / (a_ms * 1e-3)},
             "stages_ms": {"quantize": q_ms, "select": s_ms, "attn_fwd": a_ms},
             "stages_gbs": {"quantize": quantize_algorithmic_bytes(w) / (q_ms * 1e-3) / 1e9,
                            "select": select_algorithmic_bytes(w) / (s_ms * 1e-3) / 1e9,
