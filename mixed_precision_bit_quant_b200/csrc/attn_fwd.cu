@@ -7,30 +7,33 @@
 // (abstract): one hybrid-precision attention operator for prefill.
 //
 // One CTA computes one 128-row query tile (b, hq, i) against the key tiles
-// j = 0 .. (causal ? i : T-1) in ascending order.  384 threads, 12 warps:
-//   warps 0-3 / 4-7  softmax groups 0 / 1; group w takes tiles j = w, w+2, ...
-//              One thread owns one query row (= TMEM lane) of its tiles: read S
-//              from TMEM once, mask edge tiles, row max, take the exact running
-//              maximum from the other group (shared memory + mbarrier), exp2,
-//              partial row sums, P (e4m3 or bf16) into TMEM, O rescaled in TMEM
-//              when a row's maximum grows.
-//   warps 8/10 TMA producers: warp 8 loads Q (NVFP4 + scales + BF16) once and
-//              per key tile NVFP4 K + scales or BF16 K; warp 10 loads e4m3 V^T or
+// j = 0 .. (causal ? i : T-1) in ascending order.  512 threads, 16 warps:
+//   warps 0-11 softmax groups 0, 1, 2 (four warps each); group g takes the tiles
+//              j = g, g+3, ...  One thread owns one query row (= TMEM lane) of its
+//              tiles: read S from TMEM once, mask edge tiles, row max, take the
+//              exact running maximum m_{j-1} from the group of tile j-1 (shared
+//              memory + mbarrier), exp2, partial row sums, P (e4m3 or bf16) into
+//              TMEM, O rescaled in TMEM when a row's maximum grows.  Three groups
+//              put three softmax warps on each SM sub-partition, so one group's
+//              exponentials run while the others load S, reduce maxima or wait.
+//   warps 12/14 TMA producers: warp 12 loads Q (NVFP4 + scales + BF16) once and
+//              per key tile NVFP4 K + scales or BF16 K; warp 14 loads e4m3 V^T or
 //              BF16 V^T, per mask bit.
-//   warp 9     TMEM allocator and QK^T issuer (one thread): FP4 pair
+//   warp 13    TMEM allocator and QK^T issuer (one thread): FP4 pair
 //              S = Q4 K4^T kind::mxf4nvf4 (block scales in TMEM), BF16 pair
-//              S = Q K^T kind::f16; S of tile j+2 as soon as group j%2 read S_j.
-//   warp 11    P.V issuer (one thread): O += P8 V8 kind::f8f6f4 or O += P16 Vs
+//              S = Q K^T kind::f16, into S buffer j % 2 as soon as S_{j-2} was read.
+//   warp 15    P.V issuer (one thread): O += P8 V8 kind::f8f6f4 or O += P16 Vs
 //              kind::f16, P read from TMEM; each product's completion is committed
 //              to a ring of mbarriers that the softmax groups wait on before
 //              they reuse a P region or rescale O.
-//   Warps 8-11 form the third warpgroup, whose registers the softmax warps
-//   take over with setmaxnreg.
+//   Warps 12-15 form the last warpgroup, whose registers the softmax warps take
+//   over with setmaxnreg.
 // The exponentials of a 32-column chunk form one branch-free block that makes
 // both P encodings (e4m3 and bf16); one copy of this block serves FP4 and BF16
 // tiles alike, which keeps the loop small enough for the instruction cache.
 // TMEM columns: S double buffer [0,256), O [256,256+D), three 32-column e4m3 P
-// regions [256+D, 352+D) (BF16 tiles keep P in their S buffer), block scales after.
+// regions [256+D, 352+D) (region j % 3 belongs to group j % 3; BF16 tiles keep P
+// in their S buffer), block scales after.
 #include <cuda.h>
 #include <stdlib.h>
 
@@ -51,8 +54,11 @@ void set_withhold_v(int tile) { g_withhold_v.store(tile < 0 ? -1 : tile, std::me
 namespace attn {
 
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s per wait: far above any legitimate wait
-constexpr int kThreads = 384;                       // 8 softmax warps + 4 producer / issuer warps
-constexpr int kSoftmaxRegs = 224, kOtherRegs = 56;  // 256*224 + 128*56 = 384*168 (the launch budget)
+constexpr int kGroups = 3;                          // softmax groups of four warps
+constexpr int kThreads = 128 * kGroups + 128;       // + 4 producer / issuer warps
+constexpr int kSoftmaxRegs = 152, kOtherRegs = 56;  // 3*128*152 + 128*56 = 512*128 (the launch budget)
+static_assert(kGroups * 128 * kSoftmaxRegs + 128 * kOtherRegs <= 65536, "register split exceeds the launch budget");
+constexpr int kPRing = 8;                           // P_FULL barriers per group
 constexpr int kMaxW = 128;                          // mask words per query tile (T <= 4096)
 
 // Operand rings: FP4 tiles use NLO slots of K (e2m1 + scales) and of V^T (e4m3);
@@ -63,17 +69,19 @@ enum Bar : int {
   Q_FULL = 0,
   KL_FULL = 1, KL_EMPTY = KL_FULL + NLO, VL_FULL = KL_EMPTY + NLO, VL_EMPTY = VL_FULL + NLO,
   KH_FULL = VL_EMPTY + NLO, KH_EMPTY = KH_FULL + NHI, VH_FULL = KH_EMPTY + NHI, VH_EMPTY = VH_FULL + NHI,
-  // P_FULL is a ring of four barriers per softmax group, indexed by the group's
-  // tile count u: a group can finish a tile before the P.V issuer has waited on
-  // the group's previous one (a BF16 tile needs no P region), so one barrier per
-  // group could complete two phases under the issuer.  Before the group finishes
-  // its tile u+3, either its FP4 tile waited for P.V up to a tile after u or a
-  // BF16 predecessor's S buffer waited for that tile's P.V, so four slots never alias.
+  // P_FULL is a ring of kPRing barriers per softmax group, indexed by the group's
+  // tile count: a group reuses a slot 3 * kPRing tiles later, so it must not run that
+  // far ahead of the P.V issuer.  It cannot: to start tile j it needed m_{j-1}, so
+  // tile j-2 had started and tile j-5 (same group) had finished; an FP4 tile j-5
+  // waited for P_{j-8} V_{j-8}, a BF16 tile j-5 made S_{j-3} wait for P_{j-5} V_{j-5}.
+  // Either way the issuer is past tile j-8 when tile j's P arrives.
   // PVC is the ring of P.V completion barriers (see pv_wait).
-  S_FULL = VH_EMPTY + NHI, S_FREE = S_FULL + 2, P_FULL = S_FREE + 2, PVC = P_FULL + 8,
+  // S_FULL is indexed by tile % 4 (three groups share the two S buffers: a group may
+  // wait for its next tile while the buffer still has the phase of the tile before)
+  S_FULL = VH_EMPTY + NHI, S_FREE = S_FULL + 4, P_FULL = S_FREE + 2, PVC = P_FULL + kPRing * kGroups,
   QK_DRAIN = PVC + 8, PV_DRAIN = QK_DRAIN + 1,
   MX = PV_DRAIN + 1,  // running-max hand-off [group][quarter]
-  NBAR = MX + 8
+  NBAR = MX + 4 * kGroups
 };
 
 __host__ __device__ constexpr int al(int x, int a) { return (x + a - 1) / a * a; }
@@ -99,9 +107,9 @@ struct Layout {
   static constexpr int OFF_MISC = OFF_BAR + 8 * NBAR;  // tmem holder, abort flag, completed-P.V count
   static constexpr int OFF_MASK = al(OFF_MISC + 16, 16);
   static constexpr int OFF_VSC = OFF_MASK + 4 * kMaxW;  // per-channel output scales
-  static constexpr int OFF_XCH = OFF_VSC + 4 * D;       // running maxima [2 groups][128 rows]
-  static constexpr int OFF_FIN = OFF_XCH + 4 * 256;     // final partial sums [2][128], maxima [2][128]
-  static constexpr int BYTES = OFF_FIN + 4 * 512;
+  static constexpr int OFF_XCH = OFF_VSC + 4 * D;       // running maxima [groups][128 rows]
+  static constexpr int OFF_FIN = OFF_XCH + 4 * 128 * kGroups;  // final partial sums [groups][128], maxima after
+  static constexpr int BYTES = OFF_FIN + 4 * 256 * kGroups;
   // request at least 116 KB so that one CTA (and its 512 TMEM columns) owns an SM
   static constexpr int DYN = (BYTES + 1024 > 116 * 1024) ? BYTES + 1024 : 116 * 1024;
   // TMEM columns
@@ -159,14 +167,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (tid == 0) {
     for (int k = 0; k < NBAR; ++k) {
-      const bool by_group = (k >= S_FREE && k < S_FREE + 2) || (k >= P_FULL && k < P_FULL + 8);
+      const bool by_group = (k >= S_FREE && k < S_FREE + 2) || (k >= P_FULL && k < P_FULL + kPRing * kGroups);
       mbar_init(BAR(k), by_group ? 4 : 1);  // softmax barriers: one arrival per warp of the group
     }
     *abort = 0;
     *reinterpret_cast<volatile uint32_t*>(smem + L::OFF_MISC + 8) = 0u;
     fence_mbar_init();
   }
-  if (warp == 9) {
+  if (warp == 4 * kGroups + 1) {
     tmem_alloc(smem_u32(tmem_holder), 512);
     tmem_relinquish();
   }
@@ -179,18 +187,19 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto is_hi = [&](int j) -> bool { return (mrow[j >> 5] >> (j & 31)) & 1u; };
   volatile int never = 0;
   // P_t V_t completion: tcgen05.commit to PVC[t % 8] (products complete in issue order).  A
-  // waiter for tile t cannot see the barrier two phases ahead: P_{t+8} comes from the group
-  // of tile t, which needs m_{t+7} from the other group, i.e. every wait for P_t V_t came first.
+  // waiter for tile t cannot see the barrier two phases ahead: P_{t+8} exists only after
+  // m_{t+7}, i.e. after tile t+7 started, so tiles t+1 (O rescale) and t+3 (P region) had
+  // finished and the QK^T issuer had passed S_{t+2}: every wait for P_t V_t came first.
   auto pv_wait = [&](int t) -> bool { return mbar_wait(BAR(PVC + (t & 7)), (t >> 3) & 1, abort, kWaitLimitNs); };
   int issued_lo = 0, issued_hi = 0;                 // loads a producer issued (drained on abort)
 
-  if (warp >= 8) {
+  if (warp >= 4 * kGroups) {
     regs_dec<kOtherRegs>();
-    if ((warp == 8 || warp == 10) && lane == 0) {
+    if ((warp == 4 * kGroups || warp == 4 * kGroups + 2) && lane == 0) {
       // ---------------------------------------------------------- producers
-      // warp 8 loads Q once and the K tiles, warp 10 the V tiles: K loads run
+      // warp 12 loads Q once and the K tiles, warp 14 the V tiles: K loads run
       // ahead of the softmax, bounded only by the QK^T that frees their stage.
-      const bool kside = (warp == 8);
+      const bool kside = (warp == 4 * kGroups);
       if (kside) {
         prefetch_tmap(&tm_qfp4); prefetch_tmap(&tm_kfp4); prefetch_tmap(&tm_qbf); prefetch_tmap(&tm_kbf);
         mbar_expect_tx(BAR(Q_FULL), L::QFP4 + L::QBF + L::SF);
@@ -238,7 +247,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       issued_lo = nlo;
       issued_hi = nhi;
-    } else if (warp == 9 && lane == 0) {
+    } else if (warp == 4 * kGroups + 1 && lane == 0) {
       // ---------------------------------------------------------- QK^T issuer
       constexpr int KB = D / 64;
       constexpr uint32_t fp4_row = D / 2;
@@ -292,13 +301,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_commit(BAR(KL_EMPTY + slot));
           ++n_lo;
         }
-        tc_commit(BAR(S_FULL + s));
+        tc_commit(BAR(S_FULL + (j & 3)));
       }
       if (!ok) raise_error(abort, 2u);
       // every tcgen05 op issued above completes before TMEM is released
       tc_commit(BAR(QK_DRAIN));
       mbar_wait(BAR(QK_DRAIN), 0, &never, kWaitLimitNs);
-    } else if (warp == 11 && lane == 0) {
+    } else if (warp == 4 * kGroups + 3 && lane == 0) {
       // ---------------------------------------------------------- P.V issuer
       // Issues P_t V_t in order, waits for its completion and publishes the count of
       // completed products, which the softmax groups and the epilogue wait on.
@@ -308,9 +317,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int t = 0; t < nj; ++t) {
         if ((t & 31) == 0) mw = mrow[t >> 5];
         const bool hi = (mw >> (t & 31)) & 1u;
-        const int s = t & 1, u = t >> 1;
+        const int s = t & 1, g = t % kGroups, u = t / kGroups;
         const int n = hi ? n_hi : n_lo, slots = hi ? NHI : NLO, slot = n % slots, use = n / slots;
-        if (!mbar_wait(BAR(P_FULL + 4 * s + (u & 3)), (u >> 2) & 1, abort, kWaitLimitNs) ||
+        if (!mbar_wait(BAR(P_FULL + kPRing * g + (u % kPRing)), (u / kPRing) & 1, abort, kWaitLimitNs) ||
             !mbar_wait(BAR((hi ? VH_FULL : VL_FULL) + slot), use & 1, abort, kWaitLimitNs)) {
           ok = false;
           break;
@@ -345,44 +354,46 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     regs_inc<kSoftmaxRegs>();
     // ------------------------------------------------------------ softmax
-    // Two groups of four warps: group wg takes the key tiles j = wg, wg+2, ... (S
-    // buffer wg) and each thread owns one query row (= TMEM lane).  The exact
+    // Three groups of four warps: group wg takes the key tiles j = wg, wg+3, ... (S
+    // buffer j % 2) and each thread owns one query row (= TMEM lane).  The exact
     // running maximum is the only sequential state across tiles: group wg writes
-    // m_j per row to shared memory and signals the other group (mbarrier) as soon
-    // as it is known, so one group's exponentials overlap the other group's loads,
-    // maxima, stores and O rescales.  Each group keeps its own partial row sum
-    // relative to the maximum of its own last tile; both are combined at the end.
+    // m_j per row to shared memory and signals the group of tile j+1 (mbarrier) as
+    // soon as it is known, so one group's exponentials overlap the other groups'
+    // loads, maxima, stores and O rescales.  Each group keeps its own partial row
+    // sum relative to the maximum of its own last tile; all are combined at the end.
     const int q4 = warp & 3, wg = warp >> 2;
     const int r = q4 * 32 + lane;  // query row within the tile == TMEM lane
     const uint32_t lane_base = (uint32_t)(q4 * 32) << 16;
     const int row_g = i * 128 + r;
-    float* mbuf = reinterpret_cast<float*>(smem + L::OFF_XCH);  // [2 groups][128 rows] running max
-    const uint32_t mx_out = BAR(MX + wg * 4 + q4), mx_in = BAR(MX + (wg ^ 1) * 4 + q4);
+    float* mbuf = reinterpret_cast<float*>(smem + L::OFF_XCH);  // [groups][128 rows] running max
+    const int wprev = (wg + kGroups - 1) % kGroups;  // the group of tile j-1
+    const uint32_t mx_out = BAR(MX + wg * 4 + q4), mx_in = BAR(MX + wprev * 4 + q4);
     const float sc_hi = p.scale_log2;
     const float sc_lo = p.scale_log2 * (p.q_gs[bhq] * p.k_gs[bhk]);
     const uint32_t p_base = tmem + lane_base + L::P_COL;
     float l = 0.0f, m_ref = -INFINITY;
     bool ok = true;
     uint32_t mw = 0;
-    for (int j = wg; j < nj; j += 2) {
-      const int u = j >> 1;
-      if ((j & 31) == wg) mw = mrow[j >> 5];  // first tile of this group in a new mask word
+    for (int j = wg; j < nj; j += kGroups) {
+      const int u = j / kGroups;  // this group's tile count
+      const int sbuf = j & 1;     // S buffer of tile j
+      mw = mrow[j >> 5];
       const bool hi = (mw >> (j & 31)) & 1u;
-      if (!__all_sync(0xffffffffu, mbar_wait(BAR(S_FULL + wg), u & 1, abort, kWaitLimitNs))) {
+      if (!__all_sync(0xffffffffu, mbar_wait(BAR(S_FULL + (j & 3)), (j >> 2) & 1, abort, kWaitLimitNs))) {
         raise_error(abort, 4u);
         ok = false;
         break;
       }
       tc_fence_after();
       uint32_t v[128];
-      const uint32_t s_addr = tmem + lane_base + L::S_COL0 + 128 * wg;
+      const uint32_t s_addr = tmem + lane_base + L::S_COL0 + 128 * sbuf;
 #pragma unroll
       for (int c4 = 0; c4 < 4; ++c4) tmem_ld32(s_addr + 32 * c4, *reinterpret_cast<uint32_t(*)[32]>(&v[32 * c4]));
       tmem_ld_wait();
       // S is in registers: its TMEM buffer may take S_{j+2}
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(BAR(S_FREE + wg));
+      if (lane == 0) mbar_arrive(BAR(S_FREE + sbuf));
       if ((p.causal && j == i) || ((j + 1) * 128 > p.N)) {  // warp-uniform: only edge tiles mask
         const int lim = min(p.causal ? row_g + 1 : p.N, p.N) - j * 128;
 #pragma unroll
@@ -409,13 +420,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float sc = hi ? sc_hi : sc_lo;
       float m_prev = -INFINITY;
       if (j > 0) {
-        // m_{j-1} from the other group's warp of the same quarter
-        if (!__all_sync(0xffffffffu, mbar_wait(mx_in, ((j - 1) >> 1) & 1, abort, kWaitLimitNs))) {
+        // m_{j-1} from the warp of the same quarter in the group of tile j-1
+        if (!__all_sync(0xffffffffu, mbar_wait(mx_in, ((j - 1) / kGroups) & 1, abort, kWaitLimitNs))) {
           raise_error(abort, 4u);
           ok = false;
           break;
         }
-        m_prev = mbuf[(wg ^ 1) * 128 + r];
+        m_prev = mbuf[wprev * 128 + r];
       }
       const float m_new = fmaxf(m_prev, mloc * sc);
       mbuf[wg * 128 + r] = m_new;
@@ -426,7 +437,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t sc2 = f2pack(sc, sc);
       const uint64_t nb2 = f2pack(8.0f - m_new, 8.0f - m_new);  // p * 2^8 = 2^(s*sc - m_new + 8)
       uint64_t acc[4] = {0, 0, 0, 0};
-      uint32_t pe_all[32];
+      if (!hi && j >= 3) {
+        // P region j % 3 (this group's own) was last read by P_{j-3} V_{j-3}, issued a
+        // whole round of tiles ago: wait until it completed
+        if (!__all_sync(0xffffffffu, pv_wait(j - 3))) {
+          raise_error(abort, 4u);
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+      }
 #pragma unroll
       for (int ch = 0; ch < 4; ++ch) {  // chunks of 32 columns
         // both P encodings for every pair (no branch in the loop: one basic block per
@@ -450,21 +470,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // BF16 P overwrites the leading columns of this tile's own S buffer (already read);
         // the e4m3 P of an FP4 tile is stored once, after its P region is free
         if (hi) tmem_st16(s_addr + 16 * ch, pb);
-#pragma unroll
-        for (int q = 0; q < 8; ++q) pe_all[8 * ch + q] = pe[q];
-      }
-      if (!hi) {
-        if (j >= 3) {
-          // P region j % 3 was last read by an earlier FP4 tile's P.V, at the latest
-          // P_{j-3} V_{j-3}: wait (after the exponentials) until that product completed
-          if (!__all_sync(0xffffffffu, pv_wait(j - 3))) {
-            raise_error(abort, 4u);
-            ok = false;
-          } else {
-            tc_fence_after();
-          }
-        }
-        if (ok) tmem_st32(p_base + 32 * (j % 3), pe_all);
+        else tmem_st8(p_base + 32 * (j % 3) + 8 * ch, pe);
       }
       if (!ok) break;
       float r0, r1, r2, r3, r4, r5, r6, r7;
@@ -502,41 +508,48 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(BAR(P_FULL + 4 * wg + (u & 3)));
+      if (lane == 0) mbar_arrive(BAR(P_FULL + kPRing * wg + (u % kPRing)));
     }
     // ---------------------------------------------------------- epilogue
-    // combine the two groups' partial row sums, then each group writes D/2 columns
+    // combine the groups' partial row sums; groups 0 and 1 write D/2 columns each
     ok = ok && __all_sync(0xffffffffu, pv_wait(nj - 1));
-    float* xl = reinterpret_cast<float*>(smem + L::OFF_FIN);  // [2][128] sums, [2][128] maxima
+    float* xl = reinterpret_cast<float*>(smem + L::OFF_FIN);  // sums [groups][128], maxima [groups][128]
     xl[wg * 128 + r] = l;
-    xl[256 + wg * 128 + r] = m_ref;
-    named_bar_sync(1 + q4, 64);
+    xl[128 * kGroups + wg * 128 + r] = m_ref;
+    named_bar_sync(1 + q4, 32 * kGroups);
     if (ok) {
       tc_fence_after();
-      const float lo_ = xl[(wg ^ 1) * 128 + r], mo_ = xl[256 + (wg ^ 1) * 128 + r];
-      const float m_fin = fmaxf(m_ref, mo_);
-      const float lt = (m_ref == -INFINITY ? 0.0f : l * ex2_approx(m_ref - m_fin)) +
-                       (mo_ == -INFINITY ? 0.0f : lo_ * ex2_approx(mo_ - m_fin));
+      float m_fin = -INFINITY;
+#pragma unroll
+      for (int g = 0; g < kGroups; ++g) m_fin = fmaxf(m_fin, xl[128 * kGroups + g * 128 + r]);
+      float lt = 0.0f;
+#pragma unroll
+      for (int g = 0; g < kGroups; ++g) {
+        const float mg = xl[128 * kGroups + g * 128 + r];
+        if (mg != -INFINITY) lt += xl[g * 128 + r] * ex2_approx(mg - m_fin);
+      }
       const float inv_l = 1.0f / lt;
-      __nv_bfloat16* orow = p.o + ((size_t)bhq * p.N + row_g) * D + (D / 2) * wg;
+      if (wg < 2) {
+        __nv_bfloat16* orow = p.o + ((size_t)bhq * p.N + row_g) * D + (D / 2) * wg;
 #pragma unroll
-      for (int c4 = 0; c4 < D / 64; ++c4) {
-        uint32_t ov[32];
-        tmem_ld32(tmem + lane_base + L::O_COL + (D / 2) * wg + 32 * c4, ov);
-        tmem_ld_wait();
-        uint32_t packed[16];
+        for (int c4 = 0; c4 < D / 64; ++c4) {
+          uint32_t ov[32];
+          tmem_ld32(tmem + lane_base + L::O_COL + (D / 2) * wg + 32 * c4, ov);
+          tmem_ld_wait();
+          uint32_t packed[16];
 #pragma unroll
-        for (int c = 0; c < 32; c += 2) {
-          const int cc = (D / 2) * wg + c4 * 32 + c;
-          const float a0 = __uint_as_float(ov[c]) * (vsc[cc] * inv_l);
-          const float a1 = __uint_as_float(ov[c + 1]) * (vsc[cc + 1] * inv_l);
-          packed[c >> 1] = cvt_bf16x2(a0, a1);
-        }
-        if (row_g < p.N) {
-          uint4* dst = reinterpret_cast<uint4*>(orow + c4 * 32);
+          for (int c = 0; c < 32; c += 2) {
+            const int cc = (D / 2) * wg + c4 * 32 + c;
+            const float a0 = __uint_as_float(ov[c]) * (vsc[cc] * inv_l);
+            const float a1 = __uint_as_float(ov[c + 1]) * (vsc[cc + 1] * inv_l);
+            packed[c >> 1] = cvt_bf16x2(a0, a1);
+          }
+          if (row_g < p.N) {
+            uint4* dst = reinterpret_cast<uint4*>(orow + c4 * 32);
 #pragma unroll
-          for (int q = 0; q < 4; ++q)
-            dst[q] = make_uint4(packed[4 * q], packed[4 * q + 1], packed[4 * q + 2], packed[4 * q + 3]);
+            for (int q = 0; q < 4; ++q)
+              dst[q] = make_uint4(packed[4 * q], packed[4 * q + 1], packed[4 * q + 2], packed[4 * q + 3]);
+          }
         }
       }
       if (wg == 0 && p.lse != nullptr && row_g < p.N)
@@ -549,15 +562,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   // ------------------------------------------------------------ teardown
   tc_fence_before();
   __syncthreads();
-  if (warp == 9) {
+  if (warp == 4 * kGroups + 1) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
-  if ((warp == 8 || warp == 10) && lane == 0 && *abort) {
+  if ((warp == 4 * kGroups || warp == 4 * kGroups + 2) && lane == 0 && *abort) {
     // every role has returned and the abort flag is final: let the copies this
     // producer issued land before the CTA's shared memory goes away (a copy that
     // was never issued times out here after a quarter of the wait limit)
-    const bool kside = (warp == 8);
+    const bool kside = (warp == 4 * kGroups);
     if (kside) mbar_wait(BAR(Q_FULL), 0, &never, kWaitLimitNs / 4);
     for (int k = 0; k < NLO && k < issued_lo; ++k) {
       const int n = issued_lo - 1 - k, slot = n % NLO;
