@@ -40,20 +40,6 @@ __device__ __forceinline__ float e4m3_mag_value(uint32_t c) {
   return __uint_as_float(((ef + 120u) << 23) | (m << 20));
 }
 
-// float -> e2m1 code.  With e = clamp(floor(log2|y|), 0, 2) the spacing is
-// 2^(e-1); q = rint(|y| / 2^(e-1)); code = min(2 e + q, 7).
-__device__ __forceinline__ uint32_t e2m1_code(float y) {
-  uint32_t s = (__float_as_uint(y) >> 28) & 0x8u;
-  float a = fabsf(y);
-  int e = (int)((__float_as_uint(a) >> 23) & 0xFF) - 127;
-  e = e < 0 ? 0 : (e > 2 ? 2 : e);
-  float q = rintf(__fmul_rn(a, pow2f(1 - e)));
-  float qc = fminf(q, 8.0f);
-  uint32_t c = (uint32_t)(2 * e) + (uint32_t)qc;
-  c = c > 7u ? 7u : c;
-  return s | c;
-}
-
 // ---------------------------------------------------------------------------
 // Shared-memory addresses, fences, mbarriers.
 // ---------------------------------------------------------------------------
@@ -368,6 +354,14 @@ __device__ __forceinline__ uint32_t cvt_e4m3x2(float lo, float hi) {
   uint16_t r;
   asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
   return (uint32_t)r;
+}
+// Two floats -> two e2m1 codes in one byte (round to nearest, ties to the even
+// code, saturating at +-6): low nibble from `lo`.
+__device__ __forceinline__ uint32_t cvt_e2m1x2(float lo, float hi) {
+  uint32_t r;
+  asm("{\n\t.reg .b8 t;\n\tcvt.rn.satfinite.e2m1x2.f32 t, %1, %2;\n\tcvt.u32.u8 %0, t;\n\t}"
+      : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
 }
 // Two floats -> packed bf16x2 (RN): low half from `lo`.
 __device__ __forceinline__ uint32_t cvt_bf16x2(float lo, float hi) {

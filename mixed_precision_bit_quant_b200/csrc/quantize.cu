@@ -78,6 +78,10 @@ __global__ void __launch_bounds__(256) amax_chan_kernel(const __nv_bfloat16* __r
 // ---------------------------------------------------------------------------
 // NVFP4 pack of Q or K.  One thread = 64 consecutive elements (4 scale blocks)
 // of one row, rows 0 .. 128*T-1 (rows >= N only clear their tensor-core scales).
+// A code is the e2m1 rounding of the correctly rounded quotient x / (s * g),
+// taken two at a time by the hardware conversion to e2m1x2: round to nearest
+// with ties to the even code, saturating at +-6, the sign kept for values that
+// round to zero -- the rounding rule of the format as this library reads it.
 // ---------------------------------------------------------------------------
 template <int D>
 __global__ void __launch_bounds__(256) nvfp4_pack_kernel(
@@ -124,9 +128,11 @@ __global__ void __launch_bounds__(256) nvfp4_pack_kernel(
     uint32_t lo = 0, hi = 0;
     if (sd > 0.0f) {
 #pragma unroll
-      for (int e = 0; e < 8; ++e) lo |= e2m1_code(__fdiv_rn(f[e], den)) << (4 * e);
+      for (int e = 0; e < 4; ++e)
+        lo |= cvt_e2m1x2(__fdiv_rn(f[2 * e], den), __fdiv_rn(f[2 * e + 1], den)) << (8 * e);
 #pragma unroll
-      for (int e = 0; e < 8; ++e) hi |= e2m1_code(__fdiv_rn(f[8 + e], den)) << (4 * e);
+      for (int e = 0; e < 4; ++e)
+        hi |= cvt_e2m1x2(__fdiv_rn(f[8 + 2 * e], den), __fdiv_rn(f[9 + 2 * e], den)) << (8 * e);
     }
     out[2 * b] = lo;
     out[2 * b + 1] = hi;
