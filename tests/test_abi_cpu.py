@@ -88,3 +88,23 @@ def test_null_and_misaligned_pointers_rejected():
     assert L.thrift_select(ctypes.byref(s), 16, 16, -1, 0, 16, None, 16, 1 << 20, None) == 1
     # null mask
     assert L.thrift_attn_fwd(ctypes.byref(s), ctypes.byref(q), 16, 16, None, 16, None, None, 0, None) == 1
+
+
+def test_maximum_sizes_on_host():
+    # the mask row of a query tile is held in shared memory: at most 4096 key tiles
+    L = mq.lib()
+    at_max = mq.make_shape(1, 1, 1, 4096 * 128, 128, True)
+    assert L.thrift_quant_bytes(ctypes.byref(at_max), 0) == 4096 * 128 * 64
+    assert L.thrift_workspace_bytes(ctypes.byref(at_max), _lib.OP_SELECT) == 4 * 4096 * 128 * 2
+    over = mq.make_shape(1, 1, 1, 4096 * 128 + 1, 128, True)
+    assert L.thrift_quant_bytes(ctypes.byref(over), 0) == 0
+    q = _lib.QuantStruct(*([16] * 11))
+    assert L.thrift_quantize(ctypes.byref(over), 16, 16, 16, ctypes.byref(q), 16, 1 << 30, None) == \
+        _lib.THRIFT_ERR_UNSUPPORTED
+    assert L.thrift_attn_fwd(ctypes.byref(over), ctypes.byref(q), 16, 16, 16, 16, None, None, 0, None) == \
+        _lib.THRIFT_ERR_UNSUPPORTED
+    # the per-head kernels put (batch, head) on grid.y: B * (Hq + Hkv) <= 65535
+    wide = mq.make_shape(1, 32768, 32768, 128, 64, False)
+    assert L.thrift_quant_bytes(ctypes.byref(wide), 0) == 0
+    ok = mq.make_shape(1, 32767, 32767, 128, 64, False)
+    assert L.thrift_quant_bytes(ctypes.byref(ok), 0) == 32767 * 128 * 32
