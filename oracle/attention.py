@@ -39,6 +39,7 @@ import math
 import numpy as np
 import torch
 
+from . import mx
 from .formats import bf16_round, e4m3_decode, e4m3_encode
 from .quantize import fp8_v_quantize, nvfp4_dequantize, nvfp4_quantize, tensor_scale
 from .select import mask_bit
@@ -57,9 +58,13 @@ class Operands:
     returns them); when it is None each head is quantised when first needed,
     with the same per-head arithmetic (query tiles use the head's tensor scale
     from the whole head and quantise only their own rows).
+
+    ``fmt = "mx"`` takes the low path's operands from the microscaling variant
+    instead (``oracle.mx``: MXFP4 Q and K, MXFP8 V; ``quant`` then holds what
+    ``oracle.mx.quantize`` returns, or None to quantise the whole problem).
     """
 
-    def __init__(self, q, k, v, quant, causal: bool, sm_scale: float = 0.0):
+    def __init__(self, q, k, v, quant, causal: bool, sm_scale: float = 0.0, fmt: str = "nvfp4"):
         self._q, self._k, self._v = q, k, v
         self.quant = quant
         self.B, self.Hq, self.N, self.d = tuple(q.shape)
@@ -70,11 +75,18 @@ class Operands:
         self.sm_scale = sm_scale if sm_scale > 0 else 1.0 / math.sqrt(self.d)
         self._qc = {}
         self._kc = {}
+        self.fmt = fmt
+        if fmt == "mx":
+            self._mx = mx.dequantized(quant if quant is not None else mx.quantize(q, k, v))
+        elif fmt != "nvfp4":
+            raise ValueError(fmt)
 
     def q_tile(self, b: int, h: int, r0: int, r1: int):
         qz = self.quant
         q_hi = _f64(self._q[b, h, r0:r1])
-        if qz is not None:
+        if self.fmt == "mx":
+            q_lo = self._mx[0][b, h, r0:r1]
+        elif qz is not None:
             q_lo = nvfp4_dequantize(qz["q_codes"][b:b + 1, h:h + 1, r0:r1], qz["q_sf"][b:b + 1, h:h + 1, r0:r1],
                                     np.asarray(qz["q_g"])[b:b + 1, h:h + 1])[0, 0]
         else:
@@ -91,6 +103,8 @@ class Operands:
 
     def kv_views(self, b: int, hk: int):
         key = (b, hk)
+        if self.fmt == "mx":
+            return _f64(self._k[b, hk]), self._mx[1][b, hk], _f64(self._v[b, hk]), self._mx[2][b, hk]
         if key not in self._kc:
             qz = self.quant
             if qz is None:
@@ -157,7 +171,7 @@ def attn_query_tile(ops: Operands, mask, b: int, h: int, i: int,
 
 
 def attn_forward(q, k, v, quant, mask, causal: bool, sm_scale: float = 0.0,
-                 sigma: int = 8, p_cast: bool = True, tiles=None):
+                 sigma: int = 8, p_cast: bool = True, tiles=None, fmt: str = "nvfp4"):
     """Full (or sampled) mixed-precision attention forward.
 
     ``quant``: the quantised operands, or None to quantise each head on demand.
@@ -166,7 +180,7 @@ def attn_forward(q, k, v, quant, mask, causal: bool, sm_scale: float = 0.0,
     rows of the output are filled (the rest stay NaN).
     Returns (O[B,Hq,N,d] float64, lse[B,Hq,N] float64).
     """
-    ops = Operands(q, k, v, quant, causal, sm_scale)
+    ops = Operands(q, k, v, quant, causal, sm_scale, fmt)
     O = np.full((ops.B, ops.Hq, ops.N, ops.d), np.nan)
     lse = np.full((ops.B, ops.Hq, ops.N), np.nan)
     if tiles is None:
