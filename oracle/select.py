@@ -29,6 +29,10 @@ j % 32 of word j // 32 set means tile pair (i, j) runs in BF16.
 Parity pins: tests/test_oracle_select.py (planted scores recover the planted
 tiles, top-k dominance, popcounts, causal emptiness, budget extremes,
 nesting of budgets, pooled means against float64 means).
+
+A second mode, ``select_vertical``, ranks the fill by column votes (HyQuant's
+vertical lines); its definition is in ``select_rows_vertical`` and its pins in
+tests/test_oracle_select_vertical.py.
 """
 from __future__ import annotations
 
@@ -133,6 +137,70 @@ def select(q, k, causal: bool, budget_bp: int, budget_tiles: int = 0, rows=None)
             sc[b, h, i] = tile_scores(qp[b:b + 1, h:h + 1, i:i + 1], kp[b:b + 1, h // G:h // G + 1], 1, 1)[0, 0, 0]
     mask, counts = select_rows(sc, causal, budget_bp, budget_tiles, rows)
     return dict(qp=qp, kp=kp, scores=sc, mask=mask, counts=counts)
+
+
+def select_rows_vertical(scores, causal: bool, budget_bp: int, budget_tiles: int):
+    """The vertical-line selection mode: scores[B,Hq,T,T] -> (mask, counts, votes).
+
+    HyQuant: Hybrid-Precision Quantization for LLM Attention (abstract) keeps
+    "vertical-line" tokens -- keys that many queries attend to -- and the local
+    window in high precision, chosen by a lightweight attention-pattern signal;
+    the page gives no formula, so this library fixes one at tile level, in
+    integers so that it is exactly reproducible:
+
+    1. every query tile i of a (batch, head) votes for the tiles the score mode
+       would add to its forced ones: its k_i - |F_i| best non-forced candidates
+       by (score desc, index asc);
+    2. votes[b, h, j] = the number of query tiles of (b, h) voting for key tile j
+       (the column-importance signal);
+    3. each query tile keeps its forced tiles (sink 0 and diagonal i) and fills
+       its budget with the non-forced candidates ranked by (votes desc, score
+       desc, index asc).
+
+    The budget k_i and the forced set are those of the score mode, so every row
+    keeps the same number of BF16 tiles in both modes.
+    """
+    scores = np.asarray(scores, dtype=F32)
+    B, H, T, _ = scores.shape
+    W = (T + 31) // 32
+    votes = np.zeros((B, H, T), dtype=np.int64)
+    plan = []
+    for b in range(B):
+        for h in range(H):
+            for i in range(T):
+                n_i = i + 1 if causal else T
+                forced = sorted({0, i} & set(range(n_i)))
+                k_i = budget_for_row(n_i, len(forced), budget_bp, budget_tiles)
+                rest = [j for j in range(n_i) if j not in forced]
+                fill = max(0, k_i - len(forced)) if k_i > 0 else 0
+                s = scores[b, h, i, rest].astype(np.float64)
+                by_score = [rest[o] for o in np.lexsort((np.asarray(rest), -s))]
+                for j in by_score[:fill]:
+                    votes[b, h, j] += 1
+                plan.append((b, h, i, k_i, forced, rest, fill))
+    mask = np.zeros((B, H, T, W), dtype=np.uint32)
+    counts = np.zeros((B, H, T), dtype=np.int32)
+    for (b, h, i, k_i, forced, rest, fill) in plan:
+        chosen = []
+        if k_i > 0:
+            chosen = list(forced)
+            s = scores[b, h, i, rest].astype(np.float64)
+            v = votes[b, h, rest].astype(np.float64)
+            order = np.lexsort((np.asarray(rest), -s, -v))   # votes desc, score desc, index asc
+            chosen += [rest[o] for o in order[:fill]]
+        for j in chosen:
+            mask[b, h, i, j // 32] |= np.uint32(1) << np.uint32(j % 32)
+        counts[b, h, i] = len(chosen)
+    return mask, counts, votes
+
+
+def select_vertical(q, k, causal: bool, budget_bp: int, budget_tiles: int = 0):
+    """Pooled scores -> BF16 tile mask in the vertical-line mode (see select_rows_vertical)."""
+    qp = pool_tiles(q)
+    kp = pool_tiles(k)
+    sc = tile_scores(qp, kp, qp.shape[1], kp.shape[1])
+    mask, counts, votes = select_rows_vertical(sc, causal, budget_bp, budget_tiles)
+    return dict(qp=qp, kp=kp, scores=sc, mask=mask, counts=counts, votes=votes)
 
 
 def mask_bit(mask, b: int, h: int, i: int, j: int) -> bool:
