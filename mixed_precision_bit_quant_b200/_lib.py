@@ -92,6 +92,42 @@ def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
     return None if t is None else t.data_ptr()
 
 
+# The C ABI takes plain pointers and reads every buffer as dense and of the size
+# its shape implies, so a strided view, another dtype, a host tensor or a buffer
+# sized for another problem would be read or written out of bounds.  These checks
+# run before any call into the library.
+def _want(t: torch.Tensor, name: str, dtype: torch.dtype, shape=None, device=None) -> None:
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name}: expected a torch.Tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name}: dtype {t.dtype}, expected {dtype}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name}: must be contiguous")
+    _on_device(t, name, device)
+
+
+def _on_device(t: torch.Tensor, name: str, device=None) -> None:
+    if t.device.type != "cuda":
+        raise ValueError(f"{name}: must be a CUDA tensor (got {t.device})")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name}: on {t.device}, expected {device}")
+
+
+def _check_qkv(q: torch.Tensor, k: torch.Tensor, v: Optional[torch.Tensor] = None) -> None:
+    if not isinstance(q, torch.Tensor) or q.dim() != 4:
+        raise ValueError("q: expected a [B, Hq, N, d] tensor")
+    if not isinstance(k, torch.Tensor) or k.dim() != 4:
+        raise ValueError("k: expected a [B, Hkv, N, d] tensor")
+    B, Hq, N, d = q.shape
+    Hkv = k.shape[1]
+    _want(q, "q", torch.bfloat16)
+    _want(k, "k", torch.bfloat16, (B, Hkv, N, d), q.device)
+    if v is not None:
+        _want(v, "v", torch.bfloat16, (B, Hkv, N, d), q.device)
+
+
 def _stream() -> int:
     return torch.cuda.current_stream().cuda_stream
 
@@ -125,6 +161,16 @@ class Quantized:
         return self.tensors[k]
 
 
+def _check_quantized(quant: "Quantized", shape: Shape, device) -> None:
+    for idx, f in enumerate(QUANT_FIELDS):
+        t = quant.tensors.get(f)
+        if t is None:
+            raise ValueError(f"quantized operands: missing {f}")
+        _want(t, f, _FIELD_DTYPES.get(f, torch.uint8), device=device)
+        if t.numel() * t.element_size() < quant_bytes(shape, idx):
+            raise ValueError(f"{f}: {t.numel() * t.element_size()} bytes, the shape needs {quant_bytes(shape, idx)}")
+
+
 def alloc_quantized(shape: Shape, device) -> Quantized:
     out = {}
     for idx, f in enumerate(QUANT_FIELDS):
@@ -144,8 +190,14 @@ def _workspace(shape: Shape, op: int, device) -> Optional[torch.Tensor]:
 def quantize(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = False,
              out: Optional[Quantized] = None, ws: Optional[torch.Tensor] = None) -> Quantized:
     """thrift_quantize: NVFP4 Q, K and FP8 V (all device tensors)."""
+    _check_qkv(q, k, v)
     shape = shape_of(q, k, causal)
-    out = out if out is not None else alloc_quantized(shape, q.device)
+    if out is None:
+        out = alloc_quantized(shape, q.device)
+    else:
+        _check_quantized(out, shape, q.device)
+    if ws is not None:
+        _want(ws, "ws", torch.uint8, device=q.device)
     ws = ws if ws is not None else _workspace(shape, OP_QUANTIZE, q.device)
     st = out.struct()
     _check(lib().thrift_quantize(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), ctypes.byref(st),
@@ -157,14 +209,21 @@ def select(q: torch.Tensor, k: torch.Tensor, causal: bool, budget_bp: int = 500,
            mask: Optional[torch.Tensor] = None, counts: Optional[torch.Tensor] = None,
            ws: Optional[torch.Tensor] = None):
     """thrift_select: returns (mask[B,Hq,T,W] int32 view of the uint32 words, counts[B,Hq,T])."""
+    _check_qkv(q, k)
     shape = shape_of(q, k, causal)
     B, Hq, N, _ = q.shape
     T = (N + 127) // 128
     W = (T + 31) // 32
     if mask is None:
         mask = torch.empty((B, Hq, T, W), dtype=torch.int32, device=q.device)
+    else:
+        _want(mask, "mask", torch.int32, (B, Hq, T, W), q.device)
     if counts is None:
         counts = torch.empty((B, Hq, T), dtype=torch.int32, device=q.device)
+    else:
+        _want(counts, "counts", torch.int32, (B, Hq, T), q.device)
+    if ws is not None:
+        _want(ws, "ws", torch.uint8, device=q.device)
     ws = ws if ws is not None else _workspace(shape, OP_SELECT, q.device)
     _check(lib().thrift_select(ctypes.byref(shape), _ptr(q), _ptr(k), int(budget_bp), int(budget_tiles),
                                _ptr(mask), _ptr(counts), _ptr(ws), 0 if ws is None else ws.numel(),
@@ -176,11 +235,20 @@ def attn_fwd(q: torch.Tensor, k: torch.Tensor, quant: Quantized, mask: torch.Ten
              softmax_scale: float = 0.0, o: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
              want_lse: bool = False):
     """thrift_attn_fwd: returns (o[B,Hq,N,d] bf16, lse[B,Hq,N] fp32 or None)."""
+    _check_qkv(q, k)
     shape = shape_of(q, k, causal, softmax_scale)
+    B, Hq, N, _ = q.shape
+    T = (N + 127) // 128
+    _check_quantized(quant, shape, q.device)
+    _want(mask, "mask", torch.int32, (B, Hq, T, (T + 31) // 32), q.device)
     if o is None:
         o = torch.empty_like(q)
+    else:
+        _want(o, "o", torch.bfloat16, tuple(q.shape), q.device)
     if lse is None and want_lse:
         lse = torch.empty(q.shape[:3], dtype=torch.float32, device=q.device)
+    elif lse is not None:
+        _want(lse, "lse", torch.float32, tuple(q.shape[:3]), q.device)
     st = quant.struct()
     _check(lib().thrift_attn_fwd(ctypes.byref(shape), ctypes.byref(st), _ptr(q), _ptr(k), _ptr(mask),
                                  _ptr(o), _ptr(lse), None, 0, _stream()), "thrift_attn_fwd")
