@@ -30,6 +30,9 @@
  *    Np = 128 * T (N padded to whole tiles).
  *  - Inputs must be finite; non-finite values give undefined results.
  *  - Supported: d in {64, 128}; Hq % Hkv == 0; 1 <= N; causal in {0, 1}.
+ *    Limits: N <= 524288 (T <= 4096: one query tile's mask row is held in
+ *    shared memory), B * Hq * T < 2^31 and B * (Hq + Hkv) <= 65535 (grid
+ *    dimensions); larger shapes return THRIFT_ERR_UNSUPPORTED.
  */
 #ifndef THRIFT_H
 #define THRIFT_H
