@@ -61,7 +61,9 @@ class Operands:
 
     ``fmt = "mx"`` takes the low path's operands from the microscaling variant
     instead (``oracle.mx``: MXFP4 Q and K, MXFP8 V; ``quant`` then holds what
-    ``oracle.mx.quantize`` returns, or None to quantise the whole problem).
+    ``oracle.mx.quantize`` returns, or None to quantise the whole problem);
+    ``fmt = "mxfp4_qk"`` takes MXFP4 Q and K but keeps V's per-channel FP8
+    (``quant`` is then None).
     """
 
     def __init__(self, q, k, v, quant, causal: bool, sm_scale: float = 0.0, fmt: str = "nvfp4"):
@@ -78,13 +80,18 @@ class Operands:
         self.fmt = fmt
         if fmt == "mx":
             self._mx = mx.dequantized(quant if quant is not None else mx.quantize(q, k, v))
+        elif fmt == "mxfp4_qk":
+            qh, kh, _ = mx.dequantized(mx.quantize(q, k, v))
+            v_code, v_exp, _ = fp8_v_quantize(v)
+            vh = e4m3_decode(v_code) * np.ldexp(1.0, np.asarray(v_exp, dtype=np.int64))[:, :, None, :]
+            self._mx = (qh, kh, vh)
         elif fmt != "nvfp4":
             raise ValueError(fmt)
 
     def q_tile(self, b: int, h: int, r0: int, r1: int):
         qz = self.quant
         q_hi = _f64(self._q[b, h, r0:r1])
-        if self.fmt == "mx":
+        if self.fmt != "nvfp4":
             q_lo = self._mx[0][b, h, r0:r1]
         elif qz is not None:
             q_lo = nvfp4_dequantize(qz["q_codes"][b:b + 1, h:h + 1, r0:r1], qz["q_sf"][b:b + 1, h:h + 1, r0:r1],
@@ -103,7 +110,7 @@ class Operands:
 
     def kv_views(self, b: int, hk: int):
         key = (b, hk)
-        if self.fmt == "mx":
+        if self.fmt != "nvfp4":
             return _f64(self._k[b, hk]), self._mx[1][b, hk], _f64(self._v[b, hk]), self._mx[2][b, hk]
         if key not in self._kc:
             qz = self.quant

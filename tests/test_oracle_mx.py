@@ -151,3 +151,21 @@ def test_mxfp4_midpoints_round_to_the_even_code():
     back = mx.mx_dequantize(codes, sc, "e2m1", axis=3).ravel() / X
     assert list(back[1:1 + len(mids)]) == want
     assert list(-back[10:10 + len(mids)]) == want
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_zero_budget_mxfp4_qk_attention_keeps_channel_fp8_values(causal):
+    # MXFP4 Q and K with V in the per-channel FP8 of the NVFP4 path: at a zero budget
+    # without P rounding, softmax attention on (MX Q, MX K, channel-FP8 V)
+    from oracle import formats, quantize as oq
+    g = torch.Generator().manual_seed(7)
+    B, Hq, Hkv, N, d = 1, 2, 1, 260, 64
+    q = torch.randn(B, Hq, N, d, generator=g).to(torch.bfloat16)
+    k = torch.randn(B, Hkv, N, d, generator=g).to(torch.bfloat16)
+    v = (torch.randn(B, Hkv, N, d, generator=g) * 3).to(torch.bfloat16)
+    qh, kh, _ = mx.dequantized(mx.quantize(q, k, v))
+    v_code, v_exp, _ = oq.fp8_v_quantize(v)
+    vh = formats.e4m3_decode(v_code) * np.ldexp(1.0, v_exp.astype(np.int64))[:, :, None, :]
+    mask = osel.select(q, k, causal, 0)["mask"]
+    O, _ = oatt.attn_forward(q, k, v, None, mask, causal, p_cast=False, fmt="mxfp4_qk")
+    assert np.abs(O - oatt.exact_attention(qh, kh, vh, causal)).max() < 1e-12
