@@ -217,3 +217,32 @@ def exact_attention(q, k, v, causal: bool, sm_scale: float = 0.0):
     P = np.exp(S)
     P = P / P.sum(axis=-1, keepdims=True)
     return np.einsum("bhnm,bhmd->bhnd", P, vv)
+
+
+def exact_attention_tiles(q, k, v, causal: bool, tiles, sm_scale: float = 0.0):
+    """Textbook softmax attention in FP64 for the rows of the given query tiles.
+
+    The same definition as ``exact_attention`` (no tiles, no quantisation,
+    one softmax per row over every visible key), restricted to the rows
+    [128 i, 128 i + 128) of each (b, h, i) in ``tiles`` so that long
+    sequences do not need the whole N x N logit matrix.  Rows outside the
+    listed tiles stay NaN.  Returns O[B, Hq, N, d] float64.
+    """
+    B, Hq, N, d = tuple(q.shape)
+    G = Hq // int(k.shape[1])
+    scale = sm_scale if sm_scale > 0 else 1.0 / math.sqrt(d)
+    O = np.full((B, Hq, N, d), np.nan)
+    for (b, h, i) in tiles:
+        r0, r1 = i * 128, min(N, (i + 1) * 128)
+        n_keys = r1 if causal else N
+        qr = _f64(q[b, h, r0:r1])
+        kk = _f64(k[b, h // G, :n_keys])
+        vv = _f64(v[b, h // G, :n_keys])
+        S = (qr @ kk.T) * scale
+        if causal:
+            rows = np.arange(r0, r1)[:, None]
+            S = np.where(np.arange(n_keys)[None, :] > rows, -np.inf, S)
+        S = S - S.max(axis=1, keepdims=True)
+        P = np.exp(S)
+        O[b, h, r0:r1] = (P / P.sum(axis=1, keepdims=True)) @ vv
+    return O

@@ -61,3 +61,61 @@ def test_oracle_snapshot_unchanged():
     with open(os.path.join(GOLDEN, "oracle_snapshot.txt")) as f:
         stored = [line.strip() for line in f if line.strip() and not line.startswith("#")]
     assert mod.snapshot_lines() == stored
+
+
+def _rational(expr: str):
+    from fractions import Fraction
+    out = Fraction(1)
+    for factor in expr.split("*"):
+        parts = factor.split("/")
+        f = Fraction(int(parts[0]))
+        for p in parts[1:]:
+            f /= int(p)
+        out *= f
+    return out
+
+
+def p_cast_problem(e_t: float):
+    """The two-key problem of p_cast_closed_forms.txt: logits (0, -t) on row 0."""
+    import torch
+    d, N = 64, 2
+    q = torch.zeros((1, 1, N, d), dtype=torch.float32)
+    k = torch.zeros((1, 1, N, d), dtype=torch.float32)
+    v = torch.zeros((1, 1, N, d), dtype=torch.float32)
+    q[0, 0, 0, 0] = 10.5
+    k[0, 0, 1, 0] = -10.5
+    v[0, 0, 0, 0] = 1.0
+    v[0, 0, 1, 1] = 1.0
+    scale = math.log(e_t) / 110.25
+    return tuple(t.to(torch.bfloat16) for t in (q, k, v)) + (scale,)
+
+
+def p_cast_cases():
+    cases = []
+    with open(os.path.join(GOLDEN, "p_cast_closed_forms.txt")) as f:
+        for line in f:
+            line = line.strip()
+            if line and not line.startswith("#"):
+                name, tile, e_t, o0, o1 = line.split()
+                cases.append((name, tile, float(e_t), _rational(o0), _rational(o1)))
+    return cases
+
+
+def test_p_cast_closed_forms():
+    import numpy as np
+    from oracle.attention import attn_forward
+    from oracle.quantize import quantize
+    cases = p_cast_cases()
+    assert [c[0] for c in cases] == ["A", "B", "C", "D"]
+    for name, tile, e_t, o0, o1 in cases:
+        q, k, v, scale = p_cast_problem(e_t)
+        qz = quantize(q, k, v)
+        # the operands are exact in both precisions: only the cast of P rounds
+        assert int(qz["q_sf"][0, 0, 0, 0]) == 0x7E and float(qz["q_g"][0, 0]) == 2.0 ** -8
+        mask = np.full((1, 1, 1, 1), 1 if tile == "bf16" else 0, dtype=np.uint32)
+        O, lse = attn_forward(q, k, v, qz, mask, False, sm_scale=scale)
+        assert abs(O[0, 0, 0, 0] - float(o0)) <= 1e-12 * float(o0), name
+        assert abs(O[0, 0, 0, 1] - float(o1)) <= 1e-12 * float(o1), name
+        assert not O[0, 0, 0, 2:].any()
+        assert np.allclose(O[0, 0, 1, :2], 0.5, rtol=0, atol=1e-15) and not O[0, 0, 1, 2:].any()
+        assert abs(lse[0, 0, 0] - math.log(1.0 + 1.0 / e_t)) < 1e-12

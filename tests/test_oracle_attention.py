@@ -157,3 +157,19 @@ def test_on_demand_quantisation_matches_full_quantisation():
     O1, l1 = attn_forward(q, k, v, qz, sel["mask"], True, tiles=tiles)
     O2, l2 = attn_forward(q, k, v, None, sel["mask"], True, tiles=tiles)
     assert np.array_equal(np.nan_to_num(O1, nan=7.0), np.nan_to_num(O2, nan=7.0))
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_exact_attention_tiles_is_exact_attention_row_by_row(causal):
+    from oracle.attention import exact_attention_tiles
+    q, k, v = _problem(N=300, seed=9)
+    ref = exact_attention(q, k, v, causal)
+    tiles = [(0, 0, 0), (0, 1, 2), (0, 3, 1)]
+    O = exact_attention_tiles(q, k, v, causal, tiles)
+    for (b, h, i) in tiles:
+        r0, r1 = i * 128, min(300, (i + 1) * 128)
+        assert np.max(np.abs(O[b, h, r0:r1] - ref[b, h, r0:r1])) < 1e-12
+    assert np.isnan(O[0, 2]).all()
+    # first row of a causal problem sees one key: its value row
+    if causal:
+        assert np.allclose(O[0, 0, 0], v.double().numpy()[0, 0, 0], atol=0)
