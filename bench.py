@@ -86,6 +86,30 @@ def attn_roofline(w: workloads.Workload, peaks: dict, key: str = "bf16_tflops"):
     return dict(flops=flops, t_roof=t, peak=flops / t, hi=hi, lo=lo, t_roof_fp4_both=t_fp4_both)
 
 
+SPEC_PEAKS_TFLOPS = {"fp4": 9000.0, "fp8": 4500.0, "bf16": 2250.0}   # B200 dense, nominal
+
+
+def attn_roofline_rates(w: workloads.Workload, p4: float, p8: float, p16: float):
+    """Roofline time of the attention kernel for explicit per-precision rates (TFLOP/s)."""
+    hi, lo = hi_lo_pairs(w)
+    F = 2.0 * 128 * 128 * w.d
+    return (lo * (F / (p4 * 1e12) + F / (p8 * 1e12)) + hi * (2 * F / (p16 * 1e12)),
+            lo * (2 * F / (p4 * 1e12)) + hi * (2 * F / (p16 * 1e12)))
+
+
+def measure_mma_rates(mq) -> dict:
+    """Dense TFLOP/s of the three tensor-core instruction forms the attention kernel issues
+    (thrift_probe_mma, one CTA per SM): NVFP4 block-scaled Q.K^T, e4m3 P.V with P in tensor
+    memory, BF16 Q.K^T, each 128 x 128 x 128 per step."""
+    out = {}
+    for name, kind, iters in (("fp4", 0, 20000), ("fp8", 1, 10000), ("bf16", 2, 4000)):
+        mq.probe_mma(kind, 128, 200)
+        r = mq.probe_mma(kind, 128, iters)
+        out[name] = r["tflops"]
+        out[name + "_flop_per_clk_per_sm"] = r["flop_per_clk_per_sm"]
+    return out
+
+
 def attn_algorithmic_bytes(w: workloads.Workload, hi: int, lo: int) -> float:
     """Compulsory HBM bytes of one attention launch (each operand read once, O written once)."""
     B, Hq, Hkv, N, d = w.B, w.Hq, w.Hkv, w.N, w.d
@@ -220,14 +244,41 @@ def oracle_sample_run(w: workloads.Workload, q, k, v, tiles):
     return dt, flops
 
 
-def cpu_baseline(w, q, k, v, n_tiles: int, seed: int = 1):
+def cpu_baseline(w, q, k, v, n_tiles: int, seed: int = 1, procs: int = 0):
+    """The oracle on sampled query tiles: one core, and (procs > 1) a spawned process pool
+    over the host's cores; the full problem's time is extrapolated from the FLOP rate."""
     tiles = workloads.sample_query_tiles(w, n_tiles, seed=seed)
     dt, flops = oracle_sample_run(w, q, k, v, tiles)
-    return {"value": flops / dt / 1e12, "unit": UNIT, "cores": 1, "kind": "oracle",
-            "sample": f"{len(tiles)} query tiles (seed {seed}) of {w.name}, each as its single-head problem: "
-                      f"pool/score/select + quantise the head + mixed attention of the tile; "
-                      f"{dt:.1f} s, single-threaded numpy (FP32 decisions, FP64 attention)",
-            "seconds": dt}
+    one = flops / dt / 1e12
+    full_flops = w.causal_adjusted_flops()
+    out = {"value": one, "unit": UNIT, "cores": 1, "kind": "oracle",
+           "sample": f"{len(tiles)} query tiles (seed {seed}) of {w.name}, each as its single-head problem: "
+                     f"pool/score/select + quantise the head + mixed attention of the tile; "
+                     f"{dt:.1f} s, single-threaded numpy (FP32 decisions, FP64 attention)",
+           "seconds": dt, "extrapolated_full_problem_s_one_core": full_flops / (one * 1e12)}
+    if procs > 1:
+        import torch.multiprocessing as tmp
+        from oracle.timing import tile_problem_time
+        G = w.Hq // w.Hkv
+        ptiles = workloads.sample_query_tiles(w, procs * 2, seed=seed + 100)
+        for t in (q, k, v):
+            t.share_memory_()        # workers receive views of the same host memory, no copies
+        jobs = [(w.causal, w.budget_bp, w.budget_tiles, q[b:b + 1, h:h + 1], k[b:b + 1, h // G:h // G + 1],
+                 v[b:b + 1, h // G:h // G + 1], i) for (b, h, i) in ptiles]
+        ctx = tmp.get_context("spawn")
+        with ctx.Pool(procs) as pool:
+            pool.map(tile_problem_time, jobs[:procs], chunksize=1)   # import and warm every worker
+            t0 = time.perf_counter()
+            res = pool.map(tile_problem_time, jobs, chunksize=1)
+            wall = time.perf_counter() - t0
+        pflops = sum(f for _, f in res)
+        allc = pflops / wall / 1e12
+        out.update({"value": allc, "cores": procs, "single_core_value": one,
+                    "sample": f"{len(jobs)} query tiles (seed {seed + 100}) of {w.name} on a spawned pool of "
+                              f"{procs} processes (one BLAS thread each), {wall:.1f} s wall; single core: "
+                              f"{len(tiles)} tiles, {dt:.1f} s",
+                    "extrapolated_full_problem_s": full_flops / (allc * 1e12)})
+    return out
 
 
 def run_reference(args, w):
@@ -280,6 +331,10 @@ def main():
     ap.add_argument("--no-clocks", action="store_true")
     ap.add_argument("--cpu-tiles", type=int, default=16)
     ap.add_argument("--ref-tiles", type=int, default=1)
+    ap.add_argument("--cpu-procs", type=int, default=-1, help="oracle pool size (-1: the host's cores, at most 32)")
+    ap.add_argument("--fmt", default="nvfp4", choices=["nvfp4", "mxfp4"])
+    ap.add_argument("--mode", default="score", choices=["score", "vertical"])
+    ap.add_argument("--no-mma-probe", action="store_true")
     args = ap.parse_args()
     w = workloads.WORKLOADS[args.workload]
     if args.budget_bp is not None:
@@ -301,7 +356,7 @@ def main():
     quant = mq.alloc_quantized(mq.shape_of(q, k, w.causal), dev)
     shape = mq.shape_of(q, k, w.causal)
     ws_q = torch.empty(max(16, mq.workspace_bytes(shape, mq.OP_QUANTIZE)), dtype=torch.uint8, device=dev)
-    ws_s = torch.empty(max(16, mq.workspace_bytes(shape, mq.OP_SELECT)), dtype=torch.uint8, device=dev)
+    ws_s = torch.empty(max(16, mq.workspace_bytes(shape, mq.OP_SELECT_VERTICAL)), dtype=torch.uint8, device=dev)
     T, W = w.T, (w.T + 31) // 32
     mask = torch.empty((w.B, w.Hq, T, W), dtype=torch.int32, device=dev)
     counts = torch.empty((w.B, w.Hq, T), dtype=torch.int32, device=dev)
@@ -315,10 +370,10 @@ def main():
     def step(m=None):
         if m is not None:
             m[0].record(stream)
-        mq.quantize(q, k, v, w.causal, out=quant, ws=ws_q)
+        mq.quantize(q, k, v, w.causal, out=quant, ws=ws_q, fmt=args.fmt)
         if m is not None:
             m[1].record(stream)
-        mq.select(q, k, w.causal, w.budget_bp, w.budget_tiles, mask=mask, counts=counts, ws=ws_s)
+        mq.select(q, k, w.causal, w.budget_bp, w.budget_tiles, mask=mask, counts=counts, ws=ws_s, mode=args.mode)
         if m is not None:
             m[2].record(stream)
         mq.attn_fwd(q, k, quant, mask, w.causal, o=o)
@@ -384,8 +439,9 @@ def main():
         out_done = [torch.cuda.Event() for _ in range(2)]
 
         def run_step(qb, kb, vb, ob):
-            mq.quantize(qb, kb, vb, w.causal, out=quant, ws=ws_q)
-            mq.select(qb, kb, w.causal, w.budget_bp, w.budget_tiles, mask=mask, counts=counts, ws=ws_s)
+            mq.quantize(qb, kb, vb, w.causal, out=quant, ws=ws_q, fmt=args.fmt)
+            mq.select(qb, kb, w.causal, w.budget_bp, w.budget_tiles, mask=mask, counts=counts, ws=ws_s,
+                      mode=args.mode)
             mq.attn_fwd(qb, kb, quant, mask, w.causal, o=ob)
 
         ke = max(3, min(10, K))
@@ -422,9 +478,26 @@ def main():
                "api": "mixed_precision_bit_quant_b200.quantize/select/attn_fwd (C ABI); pinned host copies "
                       "on their own streams, overlapping the neighbouring steps' kernels"}
 
+    # tcgen05 rates of this GPU (after the timed region: the probe's launches are not counted)
+    mma = None
+    if not args.no_mma_probe:
+        mma = measure_mma_rates(mq)
+    spec_t, spec_t_fp4 = attn_roofline_rates(w, SPEC_PEAKS_TFLOPS["fp4"], SPEC_PEAKS_TFLOPS["fp8"],
+                                             SPEC_PEAKS_TFLOPS["bf16"])
+    roof_extra = {"frac_vs_spec_peaks": spec_t / (a_ms * 1e-3),
+                  "frac_vs_spec_peaks_pv_at_fp4_rate": spec_t_fp4 / (a_ms * 1e-3),
+                  "spec_peaks_tflops": SPEC_PEAKS_TFLOPS}
+    if mma is not None:
+        mt, mt_fp4 = attn_roofline_rates(w, mma["fp4"], mma["fp8"], mma["bf16"])
+        roof_extra.update({"frac_vs_tcgen05_measured": mt / (a_ms * 1e-3),
+                           "frac_vs_tcgen05_measured_pv_at_fp4_rate": mt_fp4 / (a_ms * 1e-3),
+                           "tcgen05_measured_tflops": mma,
+                           "t_roof_tcgen05_measured_ms": mt * 1e3})
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline(w, q_h, k_h, v_h, args.cpu_tiles)
+        procs = args.cpu_procs if args.cpu_procs > 0 else min(32, os.cpu_count() or 1)
+        cpu = cpu_baseline(w, q_h, k_h, v_h, args.cpu_tiles, procs=procs)
 
     traffic = None
     if w.name == "llm32k" and w.budget_bp == 500:
@@ -435,13 +508,14 @@ def main():
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
             "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "nvfp4/e4m3/bf16 (fp32 accumulate)", "data": "synthetic", "config": config_of(w, world),
+            "dtype": f"{args.fmt}/e4m3/bf16 (fp32 accumulate)", "data": "synthetic",
+            "config": dict(config_of(w, world), fmt=args.fmt, select_mode=args.mode),
             "roofline": {"bound": "tensor", "kernel": "attn_fwd_kernel<128>", "achieved": achieved, "peak": peak,
                          "unit": "TFLOP/s", "frac": achieved / peak, "traffic": traffic,
                          "peak_source": f"{peak_src} bf16 {peaks['bf16_tflops']} TF/s burst; FP8 = 2x, FP4 = 4x "
                                         f"(nominal dense ratios); BF16 pairs {roof['hi']}, FP4 pairs {roof['lo']}",
                          "t_roof_ms": roof["t_roof"] * 1e3, "algorithmic_flops": roof["flops"],
-                         "frac_if_pv_at_fp4_rate": roof["t_roof_fp4_both"] / (a_ms * 1e-3)},
+                         "frac_if_pv_at_fp4_rate": roof["t_roof_fp4_both"] / (a_ms * 1e-3), **roof_extra},
             "stages_ms": {"quantize": q_ms, "select": s_ms, "attn_fwd": a_ms},
             "stages_gbs": {"quantize": quantize_algorithmic_bytes(w) / (q_ms * 1e-3) / 1e9,
                            "select": select_algorithmic_bytes(w) / (s_ms * 1e-3) / 1e9,

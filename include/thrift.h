@@ -104,7 +104,10 @@ enum {
 };
 
 /* Operation indices for thrift_workspace_bytes. */
-enum { THRIFT_OP_QUANTIZE = 0, THRIFT_OP_SELECT = 1, THRIFT_OP_ATTN = 2 };
+enum {
+  THRIFT_OP_QUANTIZE = 0, THRIFT_OP_SELECT = 1, THRIFT_OP_ATTN = 2, THRIFT_OP_SELECT_VERTICAL = 3,
+  THRIFT_OP_QUANTIZE_MX = 4
+};
 
 /* Bytes of one thrift_quant field for `shape` (0 for a bad shape or index). */
 THRIFT_API size_t thrift_quant_bytes(const thrift_shape *shape, int field);
@@ -121,6 +124,29 @@ THRIFT_API size_t thrift_workspace_bytes(const thrift_shape *shape, int op);
 THRIFT_API thrift_status thrift_quantize(const thrift_shape *shape, const void *q, const void *k,
                               const void *v, const thrift_quant *out, void *ws,
                               size_t ws_bytes, void *stream);
+
+/*
+ * Stage 0, microscaling variant: Q and K in MXFP4 instead of NVFP4.  The
+ * attention-quantization topic page lists MXFP4 beside NVFP4 (and a
+ * diagonal-tiled mixed-precision MXFP method); the format is the OCP
+ * microscaling one: per 32 consecutive elements along d one e8m0 scale
+ * 2^e, e = floor(log2 amax_block) - 2 clamped to [-127, 127] (-127 for an
+ * all-zero block), codes e2m1(x * 2^-e) rounded to nearest, ties to the even
+ * code, saturating at +-6, sign kept; no tensor scale.  V is quantised exactly
+ * as by thrift_quantize (per-channel FP8).  Field use (buffers sized by
+ * thrift_quant_bytes, as for NVFP4):
+ *   q_fp4 / k_fp4   [B][H][N][d/2] e2m1 codes, element 2t in the low nibble;
+ *   q_sf / k_sf     [B][H][N][d/32] e8m0 codes (the first half of the buffer);
+ *   q_sf_mma / k_sf_mma [B][H][T][d/64][512]: per 64 elements of d a chunk whose
+ *                   word 16*(r%32) + 4*(r/32) holds row r's two block scales of
+ *                   that step in bytes 0 and 1 (bytes 2 and 3 zero; rows >= N 0);
+ *   q_gs / k_gs     1.0f.
+ * ws: thrift_workspace_bytes(shape, THRIFT_OP_QUANTIZE_MX) bytes (V's per-channel
+ * amax, cleared by this call).  Read these operands with thrift_attn_fwd_mx.
+ */
+THRIFT_API thrift_status thrift_quantize_mx(const thrift_shape *shape, const void *q, const void *k,
+                                            const void *v, const thrift_quant *out, void *ws,
+                                            size_t ws_bytes, void *stream);
 
 /*
  * thrift_quantize without a workspace argument.  The pages have no
@@ -168,6 +194,24 @@ THRIFT_API thrift_status thrift_select(const thrift_shape *shape, const void *q,
                             int32_t *counts, void *ws, size_t ws_bytes, void *stream);
 
 /*
+ * Stage 1, vertical-line mode.  HyQuant: Hybrid-Precision Quantization for
+ * LLM Attention (abstract) keeps "vertical-line" keys -- the ones many queries
+ * attend to -- and the local window in high precision, chosen by a light
+ * attention-pattern signal the page does not define.  This library's signal,
+ * at tile level and in integers: every query tile of a (b, hq) votes for the
+ * tiles thrift_select would add to its forced ones; a key tile's vote count is
+ * its column importance; each query tile then keeps its forced tiles (sink 0,
+ * diagonal i) and fills the same budget k_i with the remaining candidates
+ * ranked by (votes descending, score descending, index ascending).
+ * Same arguments, layouts and budget rule as thrift_select; ws must hold
+ * thrift_workspace_bytes(shape, THRIFT_OP_SELECT_VERTICAL) bytes (pooled
+ * means, then the int32 votes [B][Hq][T], cleared by this call).
+ */
+THRIFT_API thrift_status thrift_select_vertical(const thrift_shape *shape, const void *q, const void *k,
+                                                int32_t budget_bp, int32_t budget_tiles, uint32_t *mask,
+                                                int32_t *counts, void *ws, size_t ws_bytes, void *stream);
+
+/*
  * Stage 2: the fused mixed-precision attention forward.
  * For each (b, hq, query tile i) and key tiles j ascending: BF16 pairs use
  * S = Q K^T * scale on the BF16 inputs; FP4 pairs use the block-scaled NVFP4
@@ -184,6 +228,75 @@ THRIFT_API thrift_status thrift_select(const thrift_shape *shape, const void *q,
 THRIFT_API thrift_status thrift_attn_fwd(const thrift_shape *shape, const thrift_quant *quant,
                               const void *q, const void *k, const uint32_t *mask,
                               void *o, float *lse, void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * Stage 2 on MXFP4 operands (written by thrift_quantize_mx): the FP4 tile
+ * pairs run kind::mxf4 block-scaled tensor-core products (e8m0 scales per 32
+ * elements); everything else -- BF16 pairs, the online softmax, the e4m3 cast
+ * of P, the FP8 P.V product, masking, GQA, outputs -- is that of
+ * thrift_attn_fwd.  Same arguments except the workspace (none).
+ */
+THRIFT_API thrift_status thrift_attn_fwd_mx(const thrift_shape *shape, const thrift_quant *quant,
+                                            const void *q, const void *k, const uint32_t *mask,
+                                            void *o, float *lse, void *stream);
+
+/* ------------------------------------------------------------------------
+ * Decode: one step of one new query token per sequence against a
+ * mixed-precision KV cache.  HyQuant: Hybrid-Precision Quantization for LLM
+ * Attention (abstract, decode stage) compresses the KV cache with the prefill
+ * operator's principle -- sink ("vertical-line") tokens and the local window
+ * in high precision, the rest low-bit -- and fuses the dequantisation into the
+ * attention.  This library's reading: every cached token is quantised on its
+ * own, as it is appended -- K as MXFP4, V as MXFP8 (e4m3), one e8m0 scale
+ * 2^e per 32 channels, e = floor(log2 amax) - emax (2 for e2m1, 8 for e4m3),
+ * clamped to [-127, 127], -127 for a zero block, elements rounded to nearest
+ * with ties to the even code and saturated, sign kept; tokens [0, 128) (the
+ * sink tile) and [L - 128, L) (the local window) are read from the BF16 cache,
+ * every other token from its quantised form; the query stays BF16; logits
+ * q . k * scale, exact softmax over all L tokens in FP32, no rounding of P.
+ * ------------------------------------------------------------------------ */
+typedef struct {
+  int32_t B, Hq, Hkv, L, d; /* L: cached tokens (>= 1); d in {64, 128}; Hq / Hkv <= 16 */
+  float softmax_scale;      /* 0 selects 1/sqrt(d) */
+} thrift_decode_shape;
+
+/* The quantised cache (device pointers, caller-owned, sizes from thrift_decode_cache_bytes). */
+typedef struct {
+  uint8_t *kc;   /* [B][Hkv][L][d/2]  e2m1 codes of K, channel 2t in the low nibble */
+  uint8_t *ksc;  /* [B][Hkv][L][d/32] e8m0 scale codes of K                        */
+  uint8_t *vc;   /* [B][Hkv][L][d]    e4m3 codes of V                              */
+  uint8_t *vsc;  /* [B][Hkv][L][d/32] e8m0 scale codes of V                        */
+} thrift_decode_cache;
+
+enum { THRIFT_DEC_KC = 0, THRIFT_DEC_KSC, THRIFT_DEC_VC, THRIFT_DEC_VSC, THRIFT_DEC_NFIELDS };
+
+/* Bytes of one thrift_decode_cache field (0 for a bad shape or index). */
+THRIFT_API size_t thrift_decode_cache_bytes(const thrift_decode_shape *shape, int field);
+
+/* Bytes of device workspace thrift_decode_step needs (the per-chunk softmax states). */
+THRIFT_API size_t thrift_decode_workspace_bytes(const thrift_decode_shape *shape);
+
+/*
+ * Quantise cache tokens [t_begin, t_end) of every (b, kv head) into `cache`
+ * (appending a token t is the call with [t, t + 1)).  k, v: the BF16 cache
+ * [B][Hkv][L][d], device.  0 <= t_begin <= t_end <= L, else
+ * THRIFT_ERR_INVALID; an empty range enqueues nothing.
+ */
+THRIFT_API thrift_status thrift_decode_quantize_cache(const thrift_decode_shape *shape, const void *k,
+                                                      const void *v, const thrift_decode_cache *cache,
+                                                      int32_t t_begin, int32_t t_end, void *stream);
+
+/*
+ * One decode step.  q: [B][Hq][d] BF16; k, v: the BF16 cache (only the sink
+ * and window rows are read); cache: its quantised form (every token outside
+ * the sink and the window must have been quantised); o: [B][Hq][d] BF16;
+ * lse: [B][Hq] FP32 natural-log log-sum-exp, or NULL; ws:
+ * thrift_decode_workspace_bytes(shape) bytes.  Query head h reads kv head
+ * h / (Hq / Hkv).  Every pointer 16-byte aligned (lse: 4).
+ */
+THRIFT_API thrift_status thrift_decode_step(const thrift_decode_shape *shape, const void *q, const void *k,
+                                            const void *v, const thrift_decode_cache *cache, void *o,
+                                            float *lse, void *ws, size_t ws_bytes, void *stream);
 
 /*
  * Synchronises `stream`, then reads and clears the library's device error
@@ -205,6 +318,24 @@ THRIFT_API thrift_status thrift_device_status(void *stream, uint32_t *detail);
  * issued from another thread.  Always returns THRIFT_OK.
  */
 THRIFT_API thrift_status thrift_debug_withhold_v_load(int32_t tile);
+
+/*
+ * Measurement utility (not part of the method): the dense rate of the three
+ * tensor-core instruction forms the attention kernel issues, for stating its
+ * roofline against measured rates.  kind 0: block-scaled NVFP4 (e2m1 x e2m1,
+ * e4m3 scales per 16), both operands in shared memory, 128 x n x 64 per
+ * instruction; kind 1: e4m3 x e4m3 with A in tensor memory, 128 x n x 32;
+ * kind 2: BF16 x BF16 from shared memory, 128 x n x 16.  n: 128 (kinds 0-2)
+ * or 256 (kinds 1, 2).  `ctas` CTAs (one per SM when ctas <= SM count) each
+ * issue `iters` steps of K = 128 into one FP32 accumulator:
+ * 2 * 128 * n * 128 * iters * ctas FLOPs.  Synchronises `stream`; *ms gets the
+ * CUDA-event time of the launch; cycles: DEVICE buffer of `ctas` uint64
+ * (8-byte aligned) receiving each CTA's clock-cycle count.  1 <= iters <= 2^22,
+ * 1 <= ctas <= 65535, else THRIFT_ERR_INVALID; other kind / n pairs
+ * THRIFT_ERR_UNSUPPORTED; a wait longer than 2 s THRIFT_ERR_TIMEOUT.
+ */
+THRIFT_API thrift_status thrift_probe_mma(int32_t kind, int32_t n, int32_t iters, int32_t ctas, float *ms,
+                                          unsigned long long *cycles, void *stream);
 
 /* Human-readable name of a status code (static storage). */
 THRIFT_API const char *thrift_status_string(thrift_status status);

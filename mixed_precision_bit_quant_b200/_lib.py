@@ -18,7 +18,8 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libthrift.so")
 
 THRIFT_OK, THRIFT_ERR_INVALID, THRIFT_ERR_UNSUPPORTED, THRIFT_ERR_CUDA, THRIFT_ERR_TIMEOUT = range(5)
-OP_QUANTIZE, OP_SELECT, OP_ATTN = range(3)
+OP_QUANTIZE, OP_SELECT, OP_ATTN, OP_SELECT_VERTICAL, OP_QUANTIZE_MX = range(5)
+FORMATS = ("nvfp4", "mxfp4")
 QUANT_FIELDS = ["q_fp4", "q_sf", "q_sf_mma", "q_gs", "k_fp4", "k_sf", "k_sf_mma", "k_gs",
                 "v_fp8t", "v_st", "v_exp"]
 _FIELD_DTYPES = {"q_gs": torch.float32, "k_gs": torch.float32, "v_st": torch.bfloat16,
@@ -39,6 +40,18 @@ class Shape(ctypes.Structure):
 
 class QuantStruct(ctypes.Structure):
     _fields_ = [(f, ctypes.c_void_p) for f in QUANT_FIELDS]
+
+
+DECODE_FIELDS = ["kc", "ksc", "vc", "vsc"]
+
+
+class DecodeShape(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int32), ("Hq", ctypes.c_int32), ("Hkv", ctypes.c_int32),
+                ("L", ctypes.c_int32), ("d", ctypes.c_int32), ("softmax_scale", ctypes.c_float)]
+
+
+class DecodeCacheStruct(ctypes.Structure):
+    _fields_ = [(f, ctypes.c_void_p) for f in DECODE_FIELDS]
 
 
 _lib: Optional[ctypes.CDLL] = None
@@ -63,6 +76,12 @@ def lib() -> ctypes.CDLL:
         L.thrift_quantize.restype = ctypes.c_int
         L.thrift_select.argtypes = [SP, P, P, I32, I32, P, P, P, S, P]
         L.thrift_select.restype = ctypes.c_int
+        L.thrift_quantize_mx.argtypes = [SP, P, P, P, QP, P, S, P]
+        L.thrift_quantize_mx.restype = ctypes.c_int
+        L.thrift_attn_fwd_mx.argtypes = [SP, QP, P, P, P, P, P, P]
+        L.thrift_attn_fwd_mx.restype = ctypes.c_int
+        L.thrift_select_vertical.argtypes = [SP, P, P, I32, I32, P, P, P, S, P]
+        L.thrift_select_vertical.restype = ctypes.c_int
         L.thrift_attn_fwd.argtypes = [SP, QP, P, P, P, P, P, P, S, P]
         L.thrift_attn_fwd.restype = ctypes.c_int
         L.thrift_device_status.argtypes = [P, ctypes.POINTER(ctypes.c_uint32)]
@@ -71,6 +90,18 @@ def lib() -> ctypes.CDLL:
         L.thrift_status_string.restype = ctypes.c_char_p
         L.thrift_debug_withhold_v_load.argtypes = [I32]
         L.thrift_debug_withhold_v_load.restype = ctypes.c_int
+        DSP = ctypes.POINTER(DecodeShape)
+        DCP = ctypes.POINTER(DecodeCacheStruct)
+        L.thrift_decode_cache_bytes.argtypes = [DSP, ctypes.c_int]
+        L.thrift_decode_cache_bytes.restype = S
+        L.thrift_decode_workspace_bytes.argtypes = [DSP]
+        L.thrift_decode_workspace_bytes.restype = S
+        L.thrift_decode_quantize_cache.argtypes = [DSP, P, P, DCP, I32, I32, P]
+        L.thrift_decode_quantize_cache.restype = ctypes.c_int
+        L.thrift_decode_step.argtypes = [DSP, P, P, P, DCP, P, P, P, S, P]
+        L.thrift_decode_step.restype = ctypes.c_int
+        L.thrift_probe_mma.argtypes = [I32, I32, I32, I32, ctypes.POINTER(ctypes.c_float), P, P]
+        L.thrift_probe_mma.restype = ctypes.c_int
         L.thrift_launch_count.argtypes = []
         L.thrift_launch_count.restype = U64
         L.thrift_version.argtypes = []
@@ -151,8 +182,9 @@ def workspace_bytes(shape: Shape, op: int) -> int:
 
 @dataclasses.dataclass
 class Quantized:
-    """The quantised operands (device tensors), in thrift_quant field order."""
+    """The quantised operands (device tensors), in thrift_quant field order, and their FP4 format."""
     tensors: dict
+    fmt: str = "nvfp4"
 
     def struct(self) -> QuantStruct:
         return QuantStruct(*[self.tensors[f].data_ptr() for f in QUANT_FIELDS])
@@ -187,28 +219,44 @@ def _workspace(shape: Shape, op: int, device) -> Optional[torch.Tensor]:
     return torch.empty(max(n, 16), dtype=torch.uint8, device=device) if n > 0 else None
 
 
+def _want_fmt(fmt: str) -> None:
+    if fmt not in FORMATS:
+        raise ValueError(f"fmt: {fmt!r}, expected one of {FORMATS}")
+
+
 def quantize(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = False,
-             out: Optional[Quantized] = None, ws: Optional[torch.Tensor] = None) -> Quantized:
-    """thrift_quantize: NVFP4 Q, K and FP8 V (all device tensors)."""
+             out: Optional[Quantized] = None, ws: Optional[torch.Tensor] = None, fmt: str = "nvfp4") -> Quantized:
+    """thrift_quantize (fmt "nvfp4") or thrift_quantize_mx (fmt "mxfp4"): FP4 Q, K and FP8 V
+    (all device tensors)."""
+    _want_fmt(fmt)
     _check_qkv(q, k, v)
     shape = shape_of(q, k, causal)
     if out is None:
         out = alloc_quantized(shape, q.device)
     else:
         _check_quantized(out, shape, q.device)
+    op = OP_QUANTIZE if fmt == "nvfp4" else OP_QUANTIZE_MX
     if ws is not None:
         _want(ws, "ws", torch.uint8, device=q.device)
-    ws = ws if ws is not None else _workspace(shape, OP_QUANTIZE, q.device)
+        if ws.numel() < workspace_bytes(shape, op):
+            raise ValueError(f"ws: {ws.numel()} bytes, the shape needs {workspace_bytes(shape, op)}")
+    ws = ws if ws is not None else _workspace(shape, op, q.device)
     st = out.struct()
-    _check(lib().thrift_quantize(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), ctypes.byref(st),
-                                 _ptr(ws), 0 if ws is None else ws.numel(), _stream()), "thrift_quantize")
+    fn = lib().thrift_quantize if fmt == "nvfp4" else lib().thrift_quantize_mx
+    _check(fn(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), ctypes.byref(st), _ptr(ws),
+              0 if ws is None else ws.numel(), _stream()),
+           "thrift_quantize" if fmt == "nvfp4" else "thrift_quantize_mx")
+    out.fmt = fmt
     return out
 
 
 def select(q: torch.Tensor, k: torch.Tensor, causal: bool, budget_bp: int = 500, budget_tiles: int = 0,
            mask: Optional[torch.Tensor] = None, counts: Optional[torch.Tensor] = None,
-           ws: Optional[torch.Tensor] = None):
-    """thrift_select: returns (mask[B,Hq,T,W] int32 view of the uint32 words, counts[B,Hq,T])."""
+           ws: Optional[torch.Tensor] = None, mode: str = "score"):
+    """thrift_select (mode "score") or thrift_select_vertical (mode "vertical"):
+    returns (mask[B,Hq,T,W] int32 view of the uint32 words, counts[B,Hq,T])."""
+    if mode not in ("score", "vertical"):
+        raise ValueError(f"mode: {mode!r}, expected 'score' or 'vertical'")
     _check_qkv(q, k)
     shape = shape_of(q, k, causal)
     B, Hq, N, _ = q.shape
@@ -222,19 +270,23 @@ def select(q: torch.Tensor, k: torch.Tensor, causal: bool, budget_bp: int = 500,
         counts = torch.empty((B, Hq, T), dtype=torch.int32, device=q.device)
     else:
         _want(counts, "counts", torch.int32, (B, Hq, T), q.device)
+    op = OP_SELECT if mode == "score" else OP_SELECT_VERTICAL
     if ws is not None:
         _want(ws, "ws", torch.uint8, device=q.device)
-    ws = ws if ws is not None else _workspace(shape, OP_SELECT, q.device)
-    _check(lib().thrift_select(ctypes.byref(shape), _ptr(q), _ptr(k), int(budget_bp), int(budget_tiles),
-                               _ptr(mask), _ptr(counts), _ptr(ws), 0 if ws is None else ws.numel(),
-                               _stream()), "thrift_select")
+    ws = ws if ws is not None else _workspace(shape, op, q.device)
+    fn = lib().thrift_select if mode == "score" else lib().thrift_select_vertical
+    _check(fn(ctypes.byref(shape), _ptr(q), _ptr(k), int(budget_bp), int(budget_tiles), _ptr(mask), _ptr(counts),
+              _ptr(ws), 0 if ws is None else ws.numel(), _stream()),
+           "thrift_select" if mode == "score" else "thrift_select_vertical")
     return mask, counts
 
 
 def attn_fwd(q: torch.Tensor, k: torch.Tensor, quant: Quantized, mask: torch.Tensor, causal: bool,
              softmax_scale: float = 0.0, o: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
              want_lse: bool = False):
-    """thrift_attn_fwd: returns (o[B,Hq,N,d] bf16, lse[B,Hq,N] fp32 or None)."""
+    """thrift_attn_fwd (NVFP4 operands) or thrift_attn_fwd_mx (MXFP4 operands, by quant.fmt):
+    returns (o[B,Hq,N,d] bf16, lse[B,Hq,N] fp32 or None)."""
+    _want_fmt(quant.fmt)
     _check_qkv(q, k)
     shape = shape_of(q, k, causal, softmax_scale)
     B, Hq, N, _ = q.shape
@@ -250,17 +302,98 @@ def attn_fwd(q: torch.Tensor, k: torch.Tensor, quant: Quantized, mask: torch.Ten
     elif lse is not None:
         _want(lse, "lse", torch.float32, tuple(q.shape[:3]), q.device)
     st = quant.struct()
-    _check(lib().thrift_attn_fwd(ctypes.byref(shape), ctypes.byref(st), _ptr(q), _ptr(k), _ptr(mask),
-                                 _ptr(o), _ptr(lse), None, 0, _stream()), "thrift_attn_fwd")
+    if quant.fmt == "nvfp4":
+        _check(lib().thrift_attn_fwd(ctypes.byref(shape), ctypes.byref(st), _ptr(q), _ptr(k), _ptr(mask),
+                                     _ptr(o), _ptr(lse), None, 0, _stream()), "thrift_attn_fwd")
+    else:
+        _check(lib().thrift_attn_fwd_mx(ctypes.byref(shape), ctypes.byref(st), _ptr(q), _ptr(k), _ptr(mask),
+                                        _ptr(o), _ptr(lse), _stream()), "thrift_attn_fwd_mx")
     return o, lse
 
 
 def attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool, budget_bp: int = 500,
-              budget_tiles: int = 0, softmax_scale: float = 0.0, want_lse: bool = False):
-    """The whole forward pass: quantize -> select -> fused mixed attention."""
-    quant = quantize(q, k, v, causal)
-    mask, _ = select(q, k, causal, budget_bp, budget_tiles)
+              budget_tiles: int = 0, softmax_scale: float = 0.0, want_lse: bool = False, mode: str = "score",
+              fmt: str = "nvfp4"):
+    """The whole forward pass: quantize (NVFP4 or MXFP4) -> select (score or vertical mode) ->
+    fused mixed attention."""
+    quant = quantize(q, k, v, causal, fmt=fmt)
+    mask, _ = select(q, k, causal, budget_bp, budget_tiles, mode=mode)
     return attn_fwd(q, k, quant, mask, causal, softmax_scale, want_lse=want_lse)
+
+
+def decode_shape(q: torch.Tensor, k: torch.Tensor, softmax_scale: float = 0.0) -> DecodeShape:
+    B, Hq, d = q.shape
+    return DecodeShape(int(B), int(Hq), int(k.shape[1]), int(k.shape[2]), int(d), float(softmax_scale))
+
+
+def _check_decode_kv(k: torch.Tensor, v: torch.Tensor) -> None:
+    if not isinstance(k, torch.Tensor) or k.dim() != 4:
+        raise ValueError("k: expected a [B, Hkv, L, d] tensor")
+    _want(k, "k", torch.bfloat16)
+    _want(v, "v", torch.bfloat16, tuple(k.shape), k.device)
+
+
+def decode_quantize_cache(k: torch.Tensor, v: torch.Tensor, cache: Optional[dict] = None, t_begin: int = 0,
+                          t_end: Optional[int] = None) -> dict:
+    """thrift_decode_quantize_cache: per-token MXFP4 K / MXFP8 V of cache rows [t_begin, t_end).
+    Returns the cache dict (kc, ksc, vc, vsc uint8 device tensors), allocated when not given."""
+    _check_decode_kv(k, v)
+    B, Hkv, L, d = k.shape
+    shape = DecodeShape(int(B), int(Hkv), int(Hkv), int(L), int(d), 0.0)
+    if cache is None:
+        cache = {}
+        for idx, f in enumerate(DECODE_FIELDS):
+            n = int(lib().thrift_decode_cache_bytes(ctypes.byref(shape), idx))
+            if n == 0:
+                raise ThriftError(THRIFT_ERR_INVALID, "thrift_decode_cache_bytes")
+            cache[f] = torch.empty(n, dtype=torch.uint8, device=k.device)
+    else:
+        for idx, f in enumerate(DECODE_FIELDS):
+            _want(cache[f], f, torch.uint8, device=k.device)
+            if cache[f].numel() < int(lib().thrift_decode_cache_bytes(ctypes.byref(shape), idx)):
+                raise ValueError(f"{f}: buffer too small for the cache shape")
+    st = DecodeCacheStruct(*[cache[f].data_ptr() for f in DECODE_FIELDS])
+    t_end = L if t_end is None else t_end
+    _check(lib().thrift_decode_quantize_cache(ctypes.byref(shape), _ptr(k), _ptr(v), ctypes.byref(st),
+                                              int(t_begin), int(t_end), _stream()), "thrift_decode_quantize_cache")
+    return cache
+
+
+def decode_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cache: dict, softmax_scale: float = 0.0,
+                o: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None, want_lse: bool = False,
+                ws: Optional[torch.Tensor] = None):
+    """thrift_decode_step: q[B,Hq,d] against the cache -> (o[B,Hq,d] bf16, lse[B,Hq] fp32 or None)."""
+    _check_decode_kv(k, v)
+    if not isinstance(q, torch.Tensor) or q.dim() != 3:
+        raise ValueError("q: expected a [B, Hq, d] tensor")
+    _want(q, "q", torch.bfloat16, device=k.device)
+    B, Hkv, L, d = k.shape
+    if q.shape[0] != B or q.shape[2] != d:
+        raise ValueError(f"q: shape {tuple(q.shape)} does not match the cache {tuple(k.shape)}")
+    shape = decode_shape(q, k, softmax_scale)
+    for idx, f in enumerate(DECODE_FIELDS):
+        _want(cache[f], f, torch.uint8, device=k.device)
+        if cache[f].numel() < int(lib().thrift_decode_cache_bytes(ctypes.byref(shape), idx)):
+            raise ValueError(f"{f}: buffer too small for the cache shape")
+    if o is None:
+        o = torch.empty_like(q)
+    else:
+        _want(o, "o", torch.bfloat16, tuple(q.shape), k.device)
+    if lse is None and want_lse:
+        lse = torch.empty(q.shape[:2], dtype=torch.float32, device=k.device)
+    elif lse is not None:
+        _want(lse, "lse", torch.float32, tuple(q.shape[:2]), k.device)
+    need = int(lib().thrift_decode_workspace_bytes(ctypes.byref(shape)))
+    if need == 0:
+        raise ThriftError(THRIFT_ERR_UNSUPPORTED, "thrift_decode_workspace_bytes")
+    if ws is None:
+        ws = torch.empty(need, dtype=torch.uint8, device=k.device)
+    else:
+        _want(ws, "ws", torch.uint8, device=k.device)
+    st = DecodeCacheStruct(*[cache[f].data_ptr() for f in DECODE_FIELDS])
+    _check(lib().thrift_decode_step(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), ctypes.byref(st), _ptr(o),
+                                    _ptr(lse), _ptr(ws), ws.numel(), _stream()), "thrift_decode_step")
+    return o, lse
 
 
 def device_status() -> tuple:
@@ -273,6 +406,22 @@ def device_status() -> tuple:
 def debug_withhold_v_load(tile: int) -> None:
     """Watchdog test hook: later attention launches skip key tile `tile`'s V load (-1: off)."""
     _check(lib().thrift_debug_withhold_v_load(int(tile)), "thrift_debug_withhold_v_load")
+
+
+def probe_mma(kind: int, n: int = 128, iters: int = 20000, ctas: Optional[int] = None) -> dict:
+    """thrift_probe_mma: dense tensor-core rate of one MMA form (kind 0 NVFP4, 1 e4m3 with A in
+    tensor memory, 2 BF16), one CTA per SM by default.  Returns TFLOP/s and cycle figures."""
+    if ctas is None:
+        ctas = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
+    cyc = torch.zeros(ctas, dtype=torch.int64, device="cuda")
+    ms = ctypes.c_float(0.0)
+    _check(lib().thrift_probe_mma(int(kind), int(n), int(iters), int(ctas), ctypes.byref(ms), cyc.data_ptr(),
+                                  _stream()), "thrift_probe_mma")
+    flops = 2.0 * 128 * n * 128 * iters * ctas
+    c = cyc.cpu().double()
+    return {"tflops": flops / (ms.value * 1e-3) / 1e12, "ms": float(ms.value),
+            "flop_per_clk_per_sm": 2.0 * 128 * n * 128 * iters / float(c.max()),
+            "cycles_max": float(c.max()), "ctas": ctas, "iters": iters}
 
 
 def launch_count() -> int:

@@ -11,7 +11,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libthrift.so")
-SOURCES = ["api.cu", "quantize.cu", "select.cu", "attn_fwd.cu"]
+SOURCES = ["api.cu", "quantize.cu", "select.cu", "attn_fwd.cu", "decode.cu", "mma_probe.cu"]
 HEADERS = ["dev.cuh", "kernels.h", os.path.join("..", "..", "include", "thrift.h")]
 
 NVCC_FLAGS = [

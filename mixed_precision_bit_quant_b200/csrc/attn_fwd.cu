@@ -60,6 +60,12 @@ constexpr int kSoftmaxRegs = 152, kOtherRegs = 56;  // 3*128*152 + 128*56 = 512*
 static_assert(kGroups * 128 * kSoftmaxRegs + 128 * kOtherRegs <= 65536, "register split exceeds the launch budget");
 constexpr int kPRing = 8;                           // P_FULL barriers per group
 constexpr int kMaxW = 128;                          // mask words per query tile (T <= 4096)
+#ifndef THRIFT_POLY_PAIRS
+#define THRIFT_POLY_PAIRS 0x0000u
+#endif
+// Element pairs (bit t of 16, for pair t mod 16 of a row) whose exponential runs on the
+// FMA pipe; the rest run on the MUFU.
+constexpr uint32_t kPolyPairs = THRIFT_POLY_PAIRS;
 
 // Operand rings: FP4 tiles use NLO slots of K (e2m1 + scales) and of V^T (e4m3);
 // BF16 tiles use NHI slots of bf16 K and V^T.  Producer and MMA issuer walk the
@@ -138,7 +144,7 @@ __device__ __forceinline__ void raise_error(volatile int* abort, uint32_t code) 
   atomicOr(&g_attn_error_word, code);
 }
 
-template <int D>
+template <int D, bool MXFP4>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_qfp4, const __grid_constant__ CUtensorMap tm_kfp4,
                     const __grid_constant__ CUtensorMap tm_qbf, const __grid_constant__ CUtensorMap tm_kbf,
@@ -294,10 +300,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int kb = 0; kb < KB; ++kb)
             tmem_cp_32x128b_x4(sfb + 4 * kb, smem_desc(sb + L::OFF_KSF + slot * L::SF + kb * 512, 16, 128, SWZ_NONE));
 #pragma unroll
-          for (int kb = 0; kb < KB; ++kb)
-            mma_nvfp4_ss(d_s, smem_desc(sb + L::OFF_QFP4 + kb * 32, 16, 8 * fp4_row, fp4_swz),
-                         smem_desc(kb_addr + kb * 32, 16, 8 * fp4_row, fp4_swz), idesc_nvfp4(128),
-                         tmem + L::SFA_COL + 4 * kb, sfb + 4 * kb, kb > 0);
+          for (int kb = 0; kb < KB; ++kb) {
+            const uint64_t ad = smem_desc(sb + L::OFF_QFP4 + kb * 32, 16, 8 * fp4_row, fp4_swz);
+            const uint64_t bd = smem_desc(kb_addr + kb * 32, 16, 8 * fp4_row, fp4_swz);
+            if constexpr (MXFP4)
+              mma_mxfp4_ss(d_s, ad, bd, idesc_mxfp4(128), tmem + L::SFA_COL + 4 * kb, sfb + 4 * kb, kb > 0);
+            else
+              mma_nvfp4_ss(d_s, ad, bd, idesc_nvfp4(128), tmem + L::SFA_COL + 4 * kb, sfb + 4 * kb, kb > 0);
+          }
           tc_commit(BAR(KL_EMPTY + slot));
           ++n_lo;
         }
@@ -447,32 +457,46 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_fence_after();
       }
+      // per chunk of 32 columns: exponentials in place (v[c] becomes p * 2^8 in FP32),
+      // then P in the tile's own precision only.  The element pairs that kPolyPairs marks
+      // run on the FMA pipe (polynomial), the others on the MUFU.
 #pragma unroll
-      for (int ch = 0; ch < 4; ++ch) {  // chunks of 32 columns
-        // both P encodings for every pair (no branch in the loop: one basic block per
-        // chunk whose pairs overlap); the store below takes the one the tile needs
-        uint32_t pb[16], pe[8];
+      for (int ch = 0; ch < 4; ++ch) {
 #pragma unroll
-        for (int t = 0; t < 16; ++t) {  // element pairs
-          const int c = 32 * ch + 2 * t;
-          const uint64_t a2 = ffma2(f2pack(__uint_as_float(v[c]), __uint_as_float(v[c + 1])), sc2, nb2);
-          float a0, a1;
-          f2unpack(a2, a0, a1);
-          const uint64_t e2 = f2pack(ex2_approx(a0), ex2_approx(a1));
+        for (int t = 16 * ch; t < 16 * ch + 16; ++t) {
+          const uint64_t y2 = ffma2(f2pack(__uint_as_float(v[2 * t]), __uint_as_float(v[2 * t + 1])), sc2, nb2);
+          uint64_t e2;
+          if ((kPolyPairs >> (t & 15)) & 1u) {
+            e2 = exp2_poly_x2(y2);
+          } else {
+            float a0, a1;
+            f2unpack(y2, a0, a1);
+            e2 = f2pack(ex2_approx(a0), ex2_approx(a1));
+          }
           acc[t & 3] = fadd2(acc[t & 3], e2);
           float e0, e1;
           f2unpack(e2, e0, e1);
-          pb[t] = cvt_bf16x2(e0, e1);
-          const uint32_t hh = cvt_e4m3x2(e0, e1);
-          if (t & 1) pe[t >> 1] = __byte_perm(pe[t >> 1], hh, 0x5410);
-          else pe[t >> 1] = hh;
+          v[2 * t] = __float_as_uint(e0);
+          v[2 * t + 1] = __float_as_uint(e1);
         }
-        // BF16 P overwrites the leading columns of this tile's own S buffer (already read);
-        // the e4m3 P of an FP4 tile is stored once, after its P region is free
-        if (hi) tmem_st16(s_addr + 16 * ch, pb);
-        else tmem_st8(p_base + 32 * (j % 3) + 8 * ch, pe);
+        if (hi) {
+          // BF16 P overwrites the leading 64 columns of this tile's own S buffer (already read)
+          uint32_t pb[16];
+#pragma unroll
+          for (int t = 0; t < 16; ++t)
+            pb[t] = cvt_bf16x2(__uint_as_float(v[32 * ch + 2 * t]), __uint_as_float(v[32 * ch + 2 * t + 1]));
+          tmem_st16(s_addr + 16 * ch, pb);
+        } else {
+          uint32_t pe[8];
+#pragma unroll
+          for (int t = 0; t < 8; ++t) {
+            const int c = 32 * ch + 4 * t;
+            pe[t] = __byte_perm(cvt_e4m3x2(__uint_as_float(v[c]), __uint_as_float(v[c + 1])),
+                                cvt_e4m3x2(__uint_as_float(v[c + 2]), __uint_as_float(v[c + 3])), 0x5410);
+          }
+          tmem_st8(p_base + 32 * (j % 3) + 8 * ch, pe);
+        }
       }
-      if (!ok) break;
       float r0, r1, r2, r3, r4, r5, r6, r7;
       f2unpack(acc[0], r0, r1);
       f2unpack(acc[1], r2, r3);
@@ -616,7 +640,7 @@ static bool make_map(CUtensorMap* m, CUtensorMapDataType dt, const void* base, u
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int D>
+template <int D, bool MXFP4>
 static int launch_d(const AttnArgs& a, cudaStream_t st) {
   using L = Layout<D>;
   const int T = (a.N + 127) / 128, W = (T + 31) / 32;
@@ -650,7 +674,7 @@ static int launch_d(const AttnArgs& a, cudaStream_t st) {
   const float scale = a.softmax_scale > 0.0f ? a.softmax_scale : 1.0f / sqrtf((float)D);
   p.scale_log2 = scale * 1.4426950408889634f;
   p.withhold_v = g_withhold_v.load(std::memory_order_relaxed);
-  auto kern = attn_fwd_kernel<D>;
+  auto kern = attn_fwd_kernel<D, MXFP4>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::DYN) != cudaSuccess)
     return THRIFT_ERR_CUDA;
   const unsigned grid = (unsigned)(BHq * (uint64_t)T);
@@ -662,8 +686,8 @@ static int launch_d(const AttnArgs& a, cudaStream_t st) {
 }  // namespace attn
 
 int launch_attn(const AttnArgs& a, cudaStream_t s) {
-  if (a.d == 128) return attn::launch_d<128>(a, s);
-  return attn::launch_d<64>(a, s);
+  if (a.mx) return a.d == 128 ? attn::launch_d<128, true>(a, s) : attn::launch_d<64, true>(a, s);
+  return a.d == 128 ? attn::launch_d<128, false>(a, s) : attn::launch_d<64, false>(a, s);
 }
 
 cudaError_t read_and_clear_device_error(cudaStream_t s, uint32_t* word) {

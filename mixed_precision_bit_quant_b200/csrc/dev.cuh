@@ -200,6 +200,11 @@ __host__ __device__ constexpr uint32_t idesc_nvfp4(int n) {
   return (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | ((128u >> 4) << 24);
 }
 
+// kind::mxf4 block-scaled, e2m1 inputs, ue8m0 scales (bit 23), 32-element blocks, K = 64 per
+// instruction; both scale-factor id fields 0: the two scales of a row sit in bytes 0 and 1
+// of its 32-bit tensor-memory word.
+__host__ __device__ constexpr uint32_t idesc_mxfp4(int n) { return idesc_nvfp4(n) | (1u << 23); }
+
 // D[tmem] (+)= A[smem] * B[smem]^T, kind::f16.
 __device__ __forceinline__ void mma_bf16_ss(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
                                             uint32_t accum) {
@@ -230,6 +235,14 @@ __device__ __forceinline__ void mma_nvfp4_ss(uint32_t d_tmem, uint64_t a, uint64
   asm volatile(
       "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.scale_vec::4X [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
+      ::"r"(d_tmem), "l"(a), "l"(b), "r"(idesc), "r"(accum), "r"(sfa_tmem), "r"(sfb_tmem) : "memory");
+}
+// D[tmem] (+)= (A .* SFA)[smem] * (B .* SFB)[smem]^T, kind::mxf4, 32-element scale blocks.
+__device__ __forceinline__ void mma_mxfp4_ss(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
+                                             uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accum) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf4.block_scale.scale_vec::2X [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
       ::"r"(d_tmem), "l"(a), "l"(b), "r"(idesc), "r"(accum), "r"(sfa_tmem), "r"(sfb_tmem) : "memory");
 }
 // Copy 32 rows x 16 bytes from shared memory to TMEM, replicated into all four lane quarters.
@@ -340,6 +353,11 @@ __device__ __forceinline__ uint64_t fmul2(uint64_t a, uint64_t b) {
   asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
   return d;
 }
+__device__ __forceinline__ uint64_t fsub2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float d;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
@@ -374,6 +392,35 @@ __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// 2^y for two lanes on the FMA pipe instead of the MUFU: y = j + f with
+// j = round(y) (adding 1.5 * 2^23 leaves round(y) in the low mantissa bits)
+// and f in [-1/2, 1/2]; 2^f from a degree-4 polynomial whose coefficients
+// minimise the relative error on that interval (Remez exchange, max relative
+// error 2.6e-6 in FP32); 2^j enters by adding j to the exponent field.
+// y is clamped to -126 first, so any finite or -inf input gives a finite
+// result (2^-126 or a value of that size for the clamped inputs).
+__device__ __forceinline__ uint64_t exp2_poly_x2(uint64_t y2) {
+  float y0, y1;
+  f2unpack(y2, y0, y1);
+  const uint64_t y = f2pack(fmaxf(y0, -126.0f), fmaxf(y1, -126.0f));
+  const uint64_t magic = f2pack(12582912.0f, 12582912.0f);
+  const uint64_t t = fadd2(y, magic);          // 1.5 * 2^23 + round(y), exact
+  const uint64_t f = fsub2(y, fsub2(t, magic));  // y - round(y), exact
+  uint64_t p = f2pack(9.570102207362652e-03f, 9.570102207362652e-03f);
+  p = ffma2(p, f, f2pack(5.591785907745361e-02f, 5.591785907745361e-02f));
+  p = ffma2(p, f, f2pack(2.402474433183670e-01f, 2.402474433183670e-01f));
+  p = ffma2(p, f, f2pack(6.931217908859253e-01f, 6.931217908859253e-01f));
+  p = ffma2(p, f, f2pack(9.999992847442627e-01f, 9.999992847442627e-01f));
+  float p0, p1, t0, t1;
+  f2unpack(p, p0, p1);
+  f2unpack(t, t0, t1);
+  // the low 9 bits of t's encoding hold round(y) (two's complement), so
+  // shifting them into the exponent field adds round(y) to p's exponent
+  const float r0 = __uint_as_float(__float_as_uint(p0) + (__float_as_uint(t0) << 23));
+  const float r1 = __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23));
+  return f2pack(r0, r1);
 }
 
 }  // namespace thrift

@@ -127,12 +127,32 @@ __global__ void __launch_bounds__(256) nvfp4_pack_kernel(
     const float den = __fmul_rn(sd, g);
     uint32_t lo = 0, hi = 0;
     if (sd > 0.0f) {
+      // The quotient x / den, correctly rounded, decides the code.  x * fl(1/den) is
+      // within 2 ulps of it; every e2m1 rounding threshold (0.25, 0.75, 1.25, 1.75,
+      // 2.5, 3.5, 5) has at most two significant bits, i.e. 21 zero low mantissa bits,
+      // so a product farther than 3 ulps from every such value rounds to the code of
+      // the exact quotient.  The few products that are that close (and no zero) take
+      // the correctly rounded division instead.
+      const float rcp = __frcp_rn(den);
+      float qv[16];
+      bool near = false;
 #pragma unroll
-      for (int e = 0; e < 4; ++e)
-        lo |= cvt_e2m1x2(__fdiv_rn(f[2 * e], den), __fdiv_rn(f[2 * e + 1], den)) << (8 * e);
+      for (int e = 0; e < 16; ++e) {
+        qv[e] = __fmul_rn(f[e], rcp);
+        const uint32_t m = __float_as_uint(qv[e]) & 0x7FFFFFFFu;
+        near |= (m != 0u) && (((m + 3u) & 0x1FFFFFu) < 7u);
+      }
+      if (near) {
 #pragma unroll
-      for (int e = 0; e < 4; ++e)
-        hi |= cvt_e2m1x2(__fdiv_rn(f[8 + 2 * e], den), __fdiv_rn(f[9 + 2 * e], den)) << (8 * e);
+        for (int e = 0; e < 16; ++e) {
+          const uint32_t m = __float_as_uint(qv[e]) & 0x7FFFFFFFu;
+          if ((m != 0u) && (((m + 3u) & 0x1FFFFFu) < 7u)) qv[e] = __fdiv_rn(f[e], den);
+        }
+      }
+#pragma unroll
+      for (int e = 0; e < 4; ++e) lo |= cvt_e2m1x2(qv[2 * e], qv[2 * e + 1]) << (8 * e);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) hi |= cvt_e2m1x2(qv[8 + 2 * e], qv[9 + 2 * e]) << (8 * e);
     }
     out[2 * b] = lo;
     out[2 * b + 1] = hi;
@@ -206,6 +226,91 @@ __global__ void __launch_bounds__(256) fp8_v_pack_kernel(
 }
 
 // ---------------------------------------------------------------------------
+// MXFP4 pack of Q or K: the microscaling variant of the low path (the
+// attention-quantization topic page lists MXFP4 beside NVFP4; the format is
+// the OCP microscaling one).  One e8m0 power-of-two scale per 32 consecutive
+// elements along d, no tensor scale (gs = 1).  Scale exponent e =
+// floor(log2 amax_block) - 2 (2 is the exponent of e2m1's largest value 6),
+// clamped to [-127, 127], -127 for an all-zero block; codes are the e2m1
+// rounding (nearest, ties to the even code, saturating, sign kept) of
+// x * 2^-e, an exact scaling.  One thread = 64 consecutive elements (two
+// blocks) of one row, rows 0 .. 128*T-1 (rows >= N only clear their
+// tensor-core scales).
+// Outputs: codes [BH][N][D/2]; sf [BH][N][D/32] e8m0 codes, row-major;
+// sf_mma [BH][T][D/64][512]: per 64 elements of d one 512-byte chunk in the
+// tensor core's scale order, word 16*(r%32) + 4*(r/32) of row r holding the
+// two block scales of that K=64 step in bytes 0 and 1 (bytes 2, 3 zero).
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ int mx_scale_exp(float amax) {
+  const uint32_t bits = __float_as_uint(amax);
+  if (bits == 0u) return -127;
+  const int ef = (int)(bits >> 23);
+  const int fl = ef > 0 ? ef - 127 : (31 - __clz((int)bits)) - 149;  // floor(log2 amax), subnormals too
+  const int e = fl - 2;
+  return e < -127 ? -127 : (e > 127 ? 127 : e);
+}
+
+template <int D>
+__global__ void __launch_bounds__(256) mxfp4_pack_kernel(
+    const __nv_bfloat16* __restrict__ x, int BH, int N, int T, uint8_t* __restrict__ codes,
+    uint8_t* __restrict__ sf, uint8_t* __restrict__ sf_mma, float* __restrict__ gs) {
+  constexpr int KB = D / 64;  // 64-element groups per row
+  const long long rows_pad = (long long)T * 128;
+  const long long item = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (item >= (long long)BH * rows_pad * KB) return;
+  const int kb = (int)(item % KB);
+  const long long rowg = item / KB;
+  const int bh = (int)(rowg / rows_pad);
+  const int row = (int)(rowg % rows_pad);
+  if (row == 0 && kb == 0) gs[bh] = 1.0f;
+  const int t = row >> 7, rr = row & 127;
+  uint32_t* mma_word = reinterpret_cast<uint32_t*>(
+      sf_mma + ((long long)(bh * T + t) * KB + kb) * 512 + (rr & 31) * 16 + (rr >> 5) * 4);
+  if (row >= N) {
+    *mma_word = 0u;
+    return;
+  }
+  const uint4* src = reinterpret_cast<const uint4*>(x + ((long long)bh * N + row) * D + kb * 64);
+  uint32_t out[8];
+  uint32_t sb[2];
+#pragma unroll
+  for (int b = 0; b < 2; ++b) {
+    float f[32];
+    float am = 0.0f;
+#pragma unroll
+    for (int v = 0; v < 4; ++v) {
+      const uint4 u = __ldg(src + 4 * b + v);
+      const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        f[8 * v + 2 * e] = __uint_as_float(w[e] << 16);
+        f[8 * v + 2 * e + 1] = __uint_as_float(w[e] & 0xFFFF0000u);
+      }
+    }
+#pragma unroll
+    for (int e = 0; e < 32; ++e) am = fmaxf(am, fabsf(f[e]));
+    const int ex = mx_scale_exp(am);
+    // 2^-ex: a normal FP32 power of two, since a BF16 block maximum gives ex <= 125
+    const float mul = __uint_as_float((uint32_t)(127 - ex) << 23);
+#pragma unroll
+    for (int w4 = 0; w4 < 4; ++w4) {
+      uint32_t word = 0;
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        word |= cvt_e2m1x2(__fmul_rn(f[8 * w4 + 2 * e], mul), __fmul_rn(f[8 * w4 + 2 * e + 1], mul)) << (8 * e);
+      out[4 * b + w4] = word;
+    }
+    sb[b] = (uint32_t)(ex + 127);
+  }
+  uint4* dst = reinterpret_cast<uint4*>(codes + ((long long)bh * N + row) * (D / 2) + kb * 32);
+  dst[0] = make_uint4(out[0], out[1], out[2], out[3]);
+  dst[1] = make_uint4(out[4], out[5], out[6], out[7]);
+  const uint32_t pair = sb[0] | (sb[1] << 8);
+  *reinterpret_cast<uint16_t*>(sf + ((long long)bh * N + row) * (D / 32) + kb * 2) = (uint16_t)pair;
+  *mma_word = pair;
+}
+
+// ---------------------------------------------------------------------------
 // Host launchers.
 // ---------------------------------------------------------------------------
 static int grid_chunks(long long work, int per_block, int cap) {
@@ -256,6 +361,39 @@ cudaError_t launch_quantize(const QuantArgs& a, cudaStream_t s) {
   return cudaGetLastError();
 }
 
+
+// MXFP4 Q and K (mxfp4_pack_kernel), V as in launch_quantize (per-channel FP8).
+// Workspace: the per-channel amax of V, B*Hkv*d words.
+cudaError_t launch_quantize_mx(const QuantArgs& a, cudaStream_t s) {
+  const int D = a.d, T = (a.N + 127) / 128;
+  const int BHq = a.B * a.Hq, BHk = a.B * a.Hkv;
+  uint32_t* amax_v = a.amax_ws;
+  cudaError_t err = cudaMemsetAsync(amax_v, 0, sizeof(uint32_t) * (size_t)BHk * D, s);
+  if (err != cudaSuccess) return err;
+  const int rpb = 512;
+  const dim3 gv((a.N + rpb - 1) / rpb, BHk);
+  const int KB = D / 64;
+  const long long itq = (long long)BHq * T * 128 * KB, itk = (long long)BHk * T * 128 * KB;
+  if (D == 128) {
+    amax_chan_kernel<128><<<gv, 256, 0, s>>>(a.v, a.N, rpb, amax_v);
+    mxfp4_pack_kernel<128><<<(unsigned)((itq + 255) / 256), 256, 0, s>>>(a.q, BHq, a.N, T, a.out.q_fp4, a.out.q_sf,
+                                                                        a.out.q_sf_mma, a.out.q_gs);
+    mxfp4_pack_kernel<128><<<(unsigned)((itk + 255) / 256), 256, 0, s>>>(a.k, BHk, a.N, T, a.out.k_fp4, a.out.k_sf,
+                                                                        a.out.k_sf_mma, a.out.k_gs);
+    fp8_v_pack_kernel<128><<<dim3(T, BHk), 256, 0, s>>>(a.v, a.N, T, amax_v, a.out.v_fp8t,
+                                                        reinterpret_cast<__nv_bfloat16*>(a.out.v_st), a.out.v_exp);
+  } else {
+    amax_chan_kernel<64><<<gv, 256, 0, s>>>(a.v, a.N, rpb, amax_v);
+    mxfp4_pack_kernel<64><<<(unsigned)((itq + 255) / 256), 256, 0, s>>>(a.q, BHq, a.N, T, a.out.q_fp4, a.out.q_sf,
+                                                                       a.out.q_sf_mma, a.out.q_gs);
+    mxfp4_pack_kernel<64><<<(unsigned)((itk + 255) / 256), 256, 0, s>>>(a.k, BHk, a.N, T, a.out.k_fp4, a.out.k_sf,
+                                                                       a.out.k_sf_mma, a.out.k_gs);
+    fp8_v_pack_kernel<64><<<dim3(T, BHk), 256, 0, s>>>(a.v, a.N, T, amax_v, a.out.v_fp8t,
+                                                       reinterpret_cast<__nv_bfloat16*>(a.out.v_st), a.out.v_exp);
+  }
+  count_launches(4);
+  return cudaGetLastError();
+}
 
 // ---------------------------------------------------------------------------
 // Workspace-free quantisation.  Some callers cannot hand the library a device

@@ -59,19 +59,90 @@ __device__ __forceinline__ uint32_t order_key(float f) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
+// The kprime-th largest of the nonzero keys key(j), j in [0, jend), found by one warp
+// with a 4-pass radix select (8-bit digits, a 256-bin histogram in shared memory):
+// returns tau = that key and need_eq = how many keys equal to tau are among the
+// kprime largest (>= 1).  kprime <= 0 gives tau = 0xFFFFFFFF, need_eq = 0.
+template <typename KeyFn>
+__device__ __forceinline__ void radix_kth(KeyFn key, int jend, int kprime, uint32_t* hist, int lane, uint32_t& tau,
+                                          int& need_eq) {
+  tau = 0xFFFFFFFFu;
+  need_eq = 0;
+  if (kprime <= 0) return;
+  uint32_t prefix = 0, pmask = 0;
+  int remaining = kprime;  // keys still to take among those matching the prefix
+#pragma unroll 1
+  for (int pass = 0; pass < 4; ++pass) {
+    const int shift = 24 - 8 * pass;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) hist[lane * 8 + q] = 0u;
+    __syncwarp();
+    for (int j = lane; j < jend; j += 32) {
+      const uint32_t k = key(j);
+      if (k != 0u && (k & pmask) == prefix) atomicAdd(&hist[(k >> shift) & 255u], 1u);
+    }
+    __syncwarp();
+    // lane l owns digits [8l, 8l+8); counts above each lane's range by a suffix scan
+    uint32_t hv[8];
+    uint32_t lsum = 0;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      hv[q] = hist[lane * 8 + q];
+      lsum += hv[q];
+    }
+    uint32_t above = lsum;  // inclusive suffix sum over lanes >= this one
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t t = __shfl_down_sync(0xffffffffu, above, o);
+      if (lane + o < 32) above += t;
+    }
+    const uint32_t above_excl = above - lsum;  // keys in higher lanes' digits
+    // the lane whose range holds the remaining-th largest key
+    const bool mine = above_excl < (uint32_t)remaining && above >= (uint32_t)remaining;
+    int digit = 0, rem_new = 0;
+    if (mine) {
+      uint32_t cum = above_excl;
+#pragma unroll
+      for (int q = 7; q >= 0; --q) {
+        if (cum + hv[q] >= (uint32_t)remaining) {
+          digit = lane * 8 + q;
+          rem_new = remaining - (int)cum;
+          break;
+        }
+        cum += hv[q];
+      }
+    }
+    const uint32_t bal = __ballot_sync(0xffffffffu, mine);
+    const int src = __ffs(bal) - 1;
+    digit = __shfl_sync(0xffffffffu, digit, src);
+    rem_new = __shfl_sync(0xffffffffu, rem_new, src);
+    prefix |= (uint32_t)digit << shift;
+    pmask |= 0xFFu << shift;
+    remaining = rem_new;
+    __syncwarp();
+  }
+  tau = prefix;
+  need_eq = remaining;
+}
+
 // Scores + selection for R consecutive query tiles of one (b, hq).
 // grid (ceil(T / R), B*Hq), 32*R threads: R warps.
 // Scores: thread t takes the key tiles j = t, t + 32R, ... and accumulates the R
 // rows' dot products together, so each pooled key column is read once per CTA.
-// Selection: warp r takes query tile i0 + r and finds the kprime-th largest
-// candidate key by a 4-pass radix select (8-bit digits, per-warp histogram in
-// shared memory); keys above it are taken, keys equal to it in ascending tile
-// order until the budget is met.  Dynamic shared memory: R * T keys (uint32).
-template <int D, int R>
+// Selection: warp r takes query tile i0 + r.
+//  VERT = false (score mode): the kprime largest candidate scores (ties by index
+//    ascending); when `votes` is not null, every tile taken besides the forced
+//    ones adds one vote to its column, votes[b, hq, j].
+//  VERT = true (vertical-line mode): the candidates ranked by (votes desc,
+//    score desc, index asc), votes from a score-mode pass: first the vote count
+//    of the kprime-th candidate, then the scores among the candidates with that
+//    count.
+// Dynamic shared memory: R * T keys (uint32).
+template <int D, int R, bool VERT>
 __global__ void __launch_bounds__(32 * R) topk_kernel(const float* __restrict__ qp, const float* __restrict__ kpT,
                                                       int Hq, int Hkv, int T, int W, int causal, int budget_bp,
                                                       int budget_tiles, uint32_t* __restrict__ mask,
-                                                      int32_t* __restrict__ counts) {
+                                                      int32_t* __restrict__ counts, int32_t* __restrict__ votes) {
   constexpr int NT = 32 * R;
   extern __shared__ uint32_t keys[];  // [R][T]
   __shared__ float qs[R][D];
@@ -130,104 +201,77 @@ __global__ void __launch_bounds__(32 * R) topk_kernel(const float* __restrict__ 
   budget(i, n_i, nf, k_i);
   const int kprime = k_i > 0 ? k_i - nf : 0;
   const uint32_t* key = keys + warp * T;
-  const int jend = causal ? n_i : T;
-  uint32_t tau = 0xFFFFFFFFu;  // no candidate key reaches it when kprime == 0
-  int need_eq = 0;
-  if (kprime > 0) {
-    uint32_t prefix = 0, pmask = 0;
-    int remaining = kprime;  // keys still to take among those matching the prefix
-#pragma unroll 1
-    for (int pass = 0; pass < 4; ++pass) {
-      const int shift = 24 - 8 * pass;
-#pragma unroll
-      for (int q = 0; q < 8; ++q) hist[warp][lane * 8 + q] = 0u;
-      __syncwarp();
-      for (int j = lane; j < jend; j += 32) {
-        const uint32_t k = key[j];
-        if (k != 0u && (k & pmask) == prefix) atomicAdd(&hist[warp][(k >> shift) & 255u], 1u);
-      }
-      __syncwarp();
-      // lane l owns digits [8l, 8l+8); counts above each lane's range by a suffix scan
-      uint32_t hv[8];
-      uint32_t lsum = 0;
-#pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        hv[q] = hist[warp][lane * 8 + q];
-        lsum += hv[q];
-      }
-      uint32_t above = lsum;  // inclusive suffix sum over lanes >= this one
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const uint32_t t = __shfl_down_sync(0xffffffffu, above, o);
-        if (lane + o < 32) above += t;
-      }
-      const uint32_t above_excl = above - lsum;  // keys in higher lanes' digits
-      // the lane whose range holds the remaining-th largest key
-      const bool mine = above_excl < (uint32_t)remaining && above >= (uint32_t)remaining;
-      int digit = 0, rem_new = 0;
-      if (mine) {
-        uint32_t cum = above_excl;
-#pragma unroll
-        for (int q = 7; q >= 0; --q) {
-          if (cum + hv[q] >= (uint32_t)remaining) {
-            digit = lane * 8 + q;
-            rem_new = remaining - (int)cum;
-            break;
-          }
-          cum += hv[q];
-        }
-      }
-      const uint32_t bal = __ballot_sync(0xffffffffu, mine);
-      const int src = __ffs(bal) - 1;
-      digit = __shfl_sync(0xffffffffu, digit, src);
-      rem_new = __shfl_sync(0xffffffffu, rem_new, src);
-      prefix |= (uint32_t)digit << shift;
-      pmask |= 0xFFu << shift;
-      remaining = rem_new;
-      __syncwarp();
-    }
-    tau = prefix;           // the kprime-th largest candidate key
-    need_eq = remaining;    // how many keys equal to tau are taken (>= 1)
+  const int jend = causal ? n_i : T;  // keys past the causal limit were never written
+  const int32_t* vrow = VERT ? votes + (long long)bhq * T : nullptr;
+  // VERT: key1(j) = votes + 1 for candidates (0 otherwise), key2(j) = the score key of the
+  // candidates whose key1 is the threshold v1
+  uint32_t v1 = 0xFFFFFFFFu;
+  int need_v = 0;
+  if (VERT) {
+    radix_kth([&](int j) -> uint32_t { return key[j] != 0u ? (uint32_t)__ldg(vrow + j) + 1u : 0u; }, jend, kprime,
+              hist[warp], lane, v1, need_v);
   }
-  // bit j set: forced tile, key above tau, or one of the first need_eq keys equal to tau
+  auto key2 = [&](int j) -> uint32_t {
+    if (j >= jend) return 0u;
+    const uint32_t k = key[j];
+    if (!VERT) return k;
+    return (k != 0u && (uint32_t)__ldg(vrow + j) + 1u == v1) ? k : 0u;
+  };
+  uint32_t tau;
+  int need_eq;
+  radix_kth(key2, jend, VERT ? need_v : kprime, hist[warp], lane, tau, need_eq);
+  // bit j set: forced tile; VERT: more votes than v1 - 1; then key above tau, or one of
+  // the first need_eq keys equal to tau in ascending tile order
   int eq_seen = 0, total = 0;
   for (int wd = 0; wd < W; ++wd) {
     const int j = wd * 32 + lane;
-    const uint32_t k = (j < jend) ? key[j] : 0u;  // keys past the causal limit were never written
+    const uint32_t k = key2(j);
     const bool eq = k != 0u && k == tau;
     const uint32_t beq = __ballot_sync(0xffffffffu, eq);
     const int before = eq_seen + __popc(beq & ((1u << lane) - 1u));
     const bool forced = k_i > 0 && j < n_i && (j == 0 || j == i);
-    const bool bit = forced || (k != 0u && k > tau && kprime > 0) || (eq && before < need_eq);
+    bool pick = (k != 0u && k > tau) || (eq && before < need_eq);
+    if (VERT && j < jend && key[j] != 0u && (uint32_t)__ldg(vrow + j) + 1u > v1) pick = true;
+    const bool bit = forced || (pick && kprime > 0);
     const uint32_t word = __ballot_sync(0xffffffffu, bit);
     if (lane == 0) mask[((long long)bhq * T + i) * W + wd] = word;
+    if (!VERT && votes != nullptr && bit && !forced) atomicAdd(votes + (long long)bhq * T + j, 1);
     eq_seen += __popc(beq);
     total += __popc(word);
   }
   if (counts != nullptr && lane == 0) counts[(long long)bhq * T + i] = total;
 }
 
-cudaError_t launch_select(const SelectArgs& a, cudaStream_t s) {
-  const int D = a.d, T = (a.N + 127) / 128, W = (T + 31) / 32;
+template <int D>
+static void launch_select_d(const SelectArgs& a, int T, int W, float* qp, float* kpT, cudaStream_t s) {
   const int BHq = a.B * a.Hq, BHk = a.B * a.Hkv;
-  float* qp = a.pool_ws;
-  float* kpT = qp + (size_t)BHq * T * D;
-  dim3 gp(T, BHq + BHk);
   constexpr int R = 8;
   const size_t dyn = (size_t)R * T * 4;
-  const dim3 gt((T + R - 1) / R, BHq);
-  if (D == 128) {
-    pool_kernel<128><<<gp, 64, 0, s>>>(a.q, a.k, BHq, a.N, T, qp, kpT);
-    if (dyn > 48 * 1024) cudaFuncSetAttribute(topk_kernel<128, R>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dyn);
-    topk_kernel<128, R><<<gt, 32 * R, dyn, s>>>(qp, kpT, a.Hq, a.Hkv, T, W, a.causal, a.budget_bp, a.budget_tiles,
-                                                a.mask, a.counts);
-  } else {
-    pool_kernel<64><<<gp, 32, 0, s>>>(a.q, a.k, BHq, a.N, T, qp, kpT);
-    if (dyn > 48 * 1024) cudaFuncSetAttribute(topk_kernel<64, R>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dyn);
-    topk_kernel<64, R><<<gt, 32 * R, dyn, s>>>(qp, kpT, a.Hq, a.Hkv, T, W, a.causal, a.budget_bp, a.budget_tiles,
-                                               a.mask, a.counts);
-  }
+  const dim3 gp(T, BHq + BHk), gt((T + R - 1) / R, BHq);
+  pool_kernel<D><<<gp, D / 2, 0, s>>>(a.q, a.k, BHq, a.N, T, qp, kpT);
+  if (dyn > 48 * 1024) cudaFuncSetAttribute(topk_kernel<D, R, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dyn);
+  topk_kernel<D, R, false><<<gt, 32 * R, dyn, s>>>(qp, kpT, a.Hq, a.Hkv, T, W, a.causal, a.budget_bp, a.budget_tiles,
+                                                   a.mask, a.counts, a.votes);
   count_launches(2);
+  if (a.vertical) {
+    if (dyn > 48 * 1024) cudaFuncSetAttribute(topk_kernel<D, R, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dyn);
+    topk_kernel<D, R, true><<<gt, 32 * R, dyn, s>>>(qp, kpT, a.Hq, a.Hkv, T, W, a.causal, a.budget_bp, a.budget_tiles,
+                                                    a.mask, a.counts, a.votes);
+    count_launches(1);
+  }
+}
+
+cudaError_t launch_select(const SelectArgs& a, cudaStream_t s) {
+  const int T = (a.N + 127) / 128, W = (T + 31) / 32;
+  const int BHq = a.B * a.Hq;
+  float* qp = a.pool_ws;
+  float* kpT = qp + (size_t)BHq * T * a.d;
+  if (a.vertical) {
+    cudaError_t err = cudaMemsetAsync(a.votes, 0, sizeof(int32_t) * (size_t)BHq * T, s);
+    if (err != cudaSuccess) return err;
+  }
+  if (a.d == 128) launch_select_d<128>(a, T, W, qp, kpT, s);
+  else launch_select_d<64>(a, T, W, qp, kpT, s);
   return cudaGetLastError();
 }
 

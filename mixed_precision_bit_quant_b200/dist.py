@@ -68,6 +68,44 @@ def shard_heads(B: int, Hq: int, Hkv: int, rank: int, world: int) -> List[Tuple[
     return out
 
 
+def shard_views(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor, rank: int, world: int):
+    """The sub-problems rank `rank` of `world` owns in one attention problem.
+
+    One (batch entry, range of kv heads) per item, with the Hq/Hkv query heads
+    of each kv head: q[b, G*h0:G*h1], k/v[b, h0:h1] and o[b, G*h0:G*h1] are
+    contiguous views of the caller's head-major tensors (no copy), and each
+    item is a complete attention problem of its own (selection, scales and
+    output are per head).  Returns a list of (q_view, k_view, v_view, o_view).
+    """
+    B, Hq, N, d = q.shape
+    Hkv = k.shape[1]
+    G = Hq // Hkv
+    out = []
+    for b, h0, h1 in shard_heads(B, Hq, Hkv, rank, world):
+        views = (q[b:b + 1, G * h0:G * h1], k[b:b + 1, h0:h1], v[b:b + 1, h0:h1], o[b:b + 1, G * h0:G * h1])
+        assert all(t.is_contiguous() for t in views)
+        out.append(views)
+    return out
+
+
+def attention_shard(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool, rank: int, world: int,
+                    budget_bp: int = 500, budget_tiles: int = 0, o: Optional[torch.Tensor] = None,
+                    mode: str = "score", fmt: str = "nvfp4") -> torch.Tensor:
+    """This rank's share of one forward pass: quantize -> select -> mixed attention on each of
+    its sub-problems (``shard_views``), written into its slices of ``o`` (allocated when None;
+    the other ranks' slices are left as they are).  No collective: a caller that wants the
+    whole O on one device gathers the slices itself.  Every rank's result equals the same
+    rows of the unsharded call bit for bit, because every quantity is per head."""
+    from . import _lib as L
+    if o is None:
+        o = torch.empty_like(q)
+    for qv, kv, vv, ov in shard_views(q, k, v, o, rank, world):
+        quant = L.quantize(qv, kv, vv, causal, fmt=fmt)
+        mask, _ = L.select(qv, kv, causal, budget_bp, budget_tiles, mode=mode)
+        L.attn_fwd(qv, kv, quant, mask, causal, o=ov)
+    return o
+
+
 def finalize() -> None:
     if dist.is_initialized():
         dist.destroy_process_group()

@@ -64,6 +64,12 @@ WORKLOADS = {
     "llm128k": Workload("llm128k", 1, 32, 8, 131072, 128, True, "llm", budget_bp=500, seed=0),
 }
 
+# A quality-axis workload with attention structure away from the sink: the
+# llm8k draw plus planted vertical lines (HyQuant: Hybrid-Precision
+# Quantization for LLM Attention, abstract: "vertical-line" tokens that many
+# queries attend to).  Not a benchmark configuration.
+VLINES = Workload("llm8k_vlines", 1, 32, 8, 8192, 128, True, "llm_vlines", budget_bp=500, seed=0)
+
 
 def custom(name: str, B: int, Hq: int, Hkv: int, N: int, d: int, causal: bool,
            kind: str = "llm", budget_bp: int = 500, budget_tiles: int = 0, seed: int = 0) -> Workload:
@@ -79,6 +85,9 @@ def generate(w: Workload, device: str = "cpu"):
           channels, drawn once, scaled by 10 in Q, K and V.
     llm:  Q, K ~ N(0,1); a per-(kv head, channel) offset ~ N(0, std 2) added
           to every key; key 0 scaled by 8 (sink); V ~ N(0,1).
+    llm_vlines: the llm draw, then per (batch, kv head) a direction u ~ N(0,1)^d:
+          16 random keys in each of 3 random key tiles (not tile 0) get + 2u and
+          every query of the group + 0.25u (planted vertical lines).
     """
     g = torch.Generator().manual_seed(w.seed)
     B, Hq, Hkv, N, d = w.B, w.Hq, w.Hkv, w.N, w.d
@@ -95,11 +104,26 @@ def generate(w: Workload, device: str = "cpu"):
         v = torch.randn((B, Hkv, N, d), generator=g, dtype=torch.float32)
         for t in (q, k, v):
             t[..., chans] *= 10.0
-    elif w.kind == "llm":
+    elif w.kind in ("llm", "llm_vlines"):
         off = 2.0 * torch.randn((B, Hkv, 1, d), generator=g, dtype=torch.float32)
         k = k + off
         k[:, :, 0, :] *= 8.0
         v = torch.randn((B, Hkv, N, d), generator=g, dtype=torch.float32)
+        if w.kind == "llm_vlines":
+            # per (batch, kv head): a direction u ~ N(0, 1)^d, 16 keys in each of 3 key
+            # tiles (never tile 0) get + 2 u, and every query of the group + 0.25 u, so those
+            # keys stand out for all queries (logit lift 0.5 |u|^2 / sqrt(d) ~ 0.5 sqrt(d))
+            T = (N + 127) // 128
+            G = Hq // Hkv
+            for b in range(B):
+                for hk in range(Hkv):
+                    u = torch.randn((d,), generator=g, dtype=torch.float32)
+                    tiles = 1 + torch.randperm(max(1, T - 1), generator=g)[:min(3, T - 1)]
+                    for t in tiles.tolist():
+                        cnt = min(128, N - 128 * t)
+                        rows = 128 * t + torch.randperm(cnt, generator=g)[:min(16, cnt)]
+                        k[b, hk, rows] += 2.0 * u
+                    q[b, G * hk:G * (hk + 1)] += 0.25 * u
     else:
         raise ValueError(f"unknown workload kind {w.kind!r}")
     out = tuple(t.to(torch.bfloat16).contiguous() for t in (q, k, v))

@@ -171,3 +171,41 @@ def test_lse_optional_and_repeatable():
     torch.cuda.synchronize()
     assert torch.equal(o1, o2)                 # deterministic
     assert lse is not None and torch.isfinite(lse).all()
+
+
+def test_p_cast_closed_forms_on_gpu():
+    """The hand-derived P-cast cases of tests/golden/p_cast_closed_forms.txt through the C ABI."""
+    from tests.test_golden import p_cast_cases, p_cast_problem
+    for name, tile, e_t, o0, o1 in p_cast_cases():
+        q, k, v, scale = p_cast_problem(e_t)
+        qd, kd, vd = _cuda(q, k, v)
+        quant = mq.quantize(qd, kd, vd)
+        mask = torch.full((1, 1, 1, 1), 1 if tile == "bf16" else 0, dtype=torch.int32, device="cuda")
+        o, _ = mq.attn_fwd(qd, kd, quant, mask, False, softmax_scale=scale)
+        st, word = mq.device_status()
+        assert st == 0, f"device watchdog raised {word:#x}"
+        og = o.float().cpu().numpy()[0, 0]
+        # only the BF16 rounding of the output separates the kernel from the closed form
+        for got, want in ((og[0, 0], float(o0)), (og[0, 1], float(o1))):
+            assert abs(got - want) <= 2.0 ** -8 * want, (name, got, want)
+        assert not og[0, 2:].any()
+        assert np.allclose(og[1, :2], 0.5, rtol=0, atol=0) and not og[1, 2:].any()
+
+
+@pytest.mark.parametrize("scale", [0.05, 0.2])
+def test_custom_softmax_scale(scale):
+    """A softmax scale other than 1/sqrt(d) on both tile kinds (the FP4 path folds the
+    tensor scales of Q and K into it)."""
+    w = workloads.custom("scale", 1, 4, 2, 700, 128, True, "llm", 3000, 0, seed=11)
+    q, k, v = workloads.generate(w)
+    qd, kd, vd = _cuda(q, k, v)
+    quant = mq.quantize(qd, kd, vd)
+    mask, _ = mq.select(qd, kd, True, 3000)
+    o, lse = mq.attn_fwd(qd, kd, quant, mask, True, softmax_scale=scale, want_lse=True)
+    st, word = mq.device_status()
+    assert st == 0, f"device watchdog raised {word:#x}"
+    ref_sel = osel.select(q, k, True, 3000)
+    assert np.array_equal(mask.cpu().numpy().view(np.uint32), ref_sel["mask"])
+    O_ref, lse_ref = oatt.attn_forward(q, k, v, None, ref_sel["mask"], True, sm_scale=scale)
+    check_close(o.float().cpu().numpy().astype(np.float64), O_ref, f"O (scale {scale})")
+    assert np.max(np.abs(lse.cpu().numpy() - lse_ref)) < 1e-3

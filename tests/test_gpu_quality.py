@@ -8,7 +8,10 @@ file measures that axis for the library's output: relative L2 and max error
 of ``thrift_attn_fwd`` (through the C ABI) against textbook attention on the
 BF16 inputs, at 0%, 5% and 100% BF16 budget, plus two controls at the 5%
 budget: the same number of BF16 tiles per query tile picked at random
-(forced sink and diagonal kept), and the forced tiles alone.
+(forced sink and diagonal kept), and the forced tiles alone; and the
+vertical-line selection mode at the same budget.  Besides the benchmark
+workloads, a llm8k draw with planted vertical lines (workloads.VLINES) puts
+attention structure away from the sink, where the selection has to find it.
 
 "Gap recovered" = (e_0 - e_5) / (e_0 - e_100) on the relative L2 error.
 
@@ -85,6 +88,9 @@ def _quality(w, tiles=None):
         o, _ = mq.attn_fwd(qd, kd, quant, mask, w.causal)
         out[f"bp{bp}"] = _err(o, ref, sel)
         if bp == 500:
+            mv, _ = mq.select(qd, kd, w.causal, bp, mode="vertical")
+            o3, _ = mq.attn_fwd(qd, kd, quant, mv, w.causal)
+            out["bp500_vertical_mode"] = _err(o3, ref, sel)
             cnt = counts.cpu().numpy()
             for name, m in (("bp500_random", _random_mask(cnt, w.causal, T, seed=7)),
                             ("forced_only", _forced_mask(cnt, w.causal, T))):
@@ -99,6 +105,7 @@ def _quality(w, tiles=None):
     out["gap_recovered"] = (e0 - e5) / (e0 - e100)
     out["gap_recovered_random"] = (e0 - out["bp500_random"]["rel_l2"]) / (e0 - e100)
     out["gap_recovered_forced_only"] = (e0 - out["forced_only"]["rel_l2"]) / (e0 - e100)
+    out["gap_recovered_vertical_mode"] = (e0 - out["bp500_vertical_mode"]["rel_l2"]) / (e0 - e100)
     out["rows"] = int(sel.sum())
     assert e100 < e0
     return out
@@ -111,6 +118,11 @@ def test_quality_llm8k_full():
 def test_quality_llm32k_sampled():
     w = workloads.WORKLOADS["llm32k"]
     _RESULTS["llm32k_64tiles"] = _quality(w, workloads.sample_query_tiles(w, 64, seed=1))
+
+
+def test_quality_llm8k_planted_vertical_lines():
+    """Structure away from the sink: the pooled score has to find the planted key tiles."""
+    _RESULTS["llm8k_vlines"] = _quality(workloads.VLINES)
 
 
 def test_quality_vit():

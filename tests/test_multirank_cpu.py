@@ -72,3 +72,42 @@ def test_reference_arm_under_two_ranks_prints_once():
     ln = lines[0]
     assert ln["impl"] == "reference" and ln["n_gpus"] == 2 and ln["value"] > 0
     assert ln["e2e"]["h2d_bytes_per_step"] == 0 and ln["cpu_baseline"]["kind"] == "oracle"
+
+
+def _shard_worker(rank, world, port, outdir):
+    """Each rank fills its shard_views slices of O with rank-specific values; a gloo
+    all-gather (test only) reassembles the whole O, which must carry every head once."""
+    import torch
+    import torch.distributed as tdist
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
+    mdist.init(None, timeout_s=60)
+    B, Hq, Hkv, N, d = 3, 8, 4, 5, 4
+    q = torch.zeros(B, Hq, N, d)
+    k = torch.zeros(B, Hkv, N, d)
+    o = torch.full((B, Hq, N, d), -1.0)
+    for qv, kv, vv, ov in mdist.shard_views(q, k, k, o, rank, world):
+        ov.fill_(float(rank))
+    parts = [torch.empty_like(o) for _ in range(world)]
+    tdist.all_gather(parts, o)
+    mdist.finalize()
+    owner = torch.full((B, Hq), -1.0)
+    for r, part in enumerate(parts):
+        mine = (part[:, :, 0, 0] == r)
+        assert bool((owner[mine] == -1).all())         # no head filled by two ranks
+        owner[mine] = r
+    with open(os.path.join(outdir, f"s{rank}.json"), "w") as f:
+        json.dump(owner.tolist(), f)
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_shard_views_partition_and_reassembly(tmp_path, world):
+    mp.start_processes(_shard_worker, args=(world, _free_port(), str(tmp_path)), nprocs=world, join=True,
+                       start_method="spawn")
+    owners = [json.load(open(tmp_path / f"s{r}.json")) for r in range(world)]
+    assert all(ow == owners[0] for ow in owners)
+    flat = [x for row in owners[0] for x in row]
+    assert -1 not in flat                                     # every head owned
+    G = 2
+    for row in owners[0]:                                     # a GQA group never splits
+        assert all(row[G * i] == row[G * i + 1] for i in range(len(row) // G))
