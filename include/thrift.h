@@ -164,7 +164,10 @@ THRIFT_API thrift_status thrift_quantize_mx(const thrift_shape *shape, const voi
  *
  * The first call on a device looks up the array's device address with that
  * device current (a one-time set-up per device); make that first call before
- * any stream capture.  All calls share the array and each clears the words it
+ * any stream capture.  The address found then is kept for the life of the
+ * process: it does not survive cudaDeviceReset or any other teardown of the
+ * device's primary context, after which this call must not be used in that
+ * process.  All calls share the array and each clears the words it
  * uses before it uses them, so calls whose work can overlap on the GPU (other
  * streams, other host threads on the same device) race on it and must be
  * serialised by the caller.

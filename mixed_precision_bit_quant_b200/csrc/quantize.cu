@@ -421,7 +421,8 @@ size_t noalloc_scratch_words() { return kNoAllocWords; }
 
 // Host code must not pass `g_noalloc_amax` itself to a kernel: on the host that
 // name is only a stand-in for the device array.  The device address is looked
-// up once per device, with that device current, on the first call made on it.
+// up once per device, with that device current, on the first call made on it,
+// and kept: it is not looked up again after a reset of the device's context.
 cudaError_t launch_quantize_noalloc(QuantArgs a, cudaStream_t s) {
   int dev = 0;
   cudaError_t err = cudaGetDevice(&dev);
