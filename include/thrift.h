@@ -259,7 +259,7 @@ THRIFT_API thrift_status thrift_attn_fwd_mx(const thrift_shape *shape, const thr
  * q . k * scale, exact softmax over all L tokens in FP32, no rounding of P.
  * ------------------------------------------------------------------------ */
 typedef struct {
-  int32_t B, Hq, Hkv, L, d; /* L: cached tokens (>= 1); d in {64, 128}; Hq / Hkv <= 16 */
+  int32_t B, Hq, Hkv, L, d; /* L: cached tokens (>= 1); d in {64, 128}; Hq / Hkv in {1, 2, 4, 8, 16} */
   float softmax_scale;      /* 0 selects 1/sqrt(d) */
 } thrift_decode_shape;
 
@@ -303,9 +303,11 @@ THRIFT_API thrift_status thrift_decode_step(const thrift_decode_shape *shape, co
 
 /*
  * Synchronises `stream`, then reads and clears the library's device error
- * word.  Returns THRIFT_ERR_TIMEOUT if a kernel's bounded wait gave up since
+ * words.  Returns THRIFT_ERR_TIMEOUT if a kernel's bounded wait gave up since
  * the last call (the kernel then returned early and its outputs are
- * undefined); *detail (if non-NULL) receives the raw error word.
+ * undefined); *detail (if non-NULL) receives the raw error word: bits 0-2
+ * from thrift_attn_fwd (1 producer, 2 tensor-core issuer, 4 softmax); the
+ * other kernels wait on nothing and set no bit.
  */
 THRIFT_API thrift_status thrift_device_status(void *stream, uint32_t *detail);
 

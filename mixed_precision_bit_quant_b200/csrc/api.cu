@@ -218,7 +218,7 @@ static int check_decode_shape(const thrift_decode_shape* s) {
   if (s->B < 1 || s->Hq < 1 || s->Hkv < 1 || s->L < 1 || s->Hq % s->Hkv != 0) return THRIFT_ERR_INVALID;
   if (!(s->softmax_scale >= 0.0f) || std::isinf(s->softmax_scale)) return THRIFT_ERR_INVALID;
   if (s->d != 64 && s->d != 128) return THRIFT_ERR_UNSUPPORTED;
-  if (s->Hq / s->Hkv > decode_max_group()) return THRIFT_ERR_UNSUPPORTED;
+  if (!decode_group_supported(s->Hq / s->Hkv)) return THRIFT_ERR_UNSUPPORTED;
   if ((long long)s->B * s->Hkv > 65535 || (long long)s->B * s->Hq > 0x7FFFFFFFLL) return THRIFT_ERR_UNSUPPORTED;
   return 0;
 }
@@ -237,7 +237,7 @@ size_t thrift_decode_cache_bytes(const thrift_decode_shape* s, int field) {
 
 size_t thrift_decode_workspace_bytes(const thrift_decode_shape* s) {
   if (check_decode_shape(s) != 0) return 0;
-  return sizeof(float) * (size_t)s->B * s->Hq * decode_nchunk(s->L) * (2 + (size_t)s->d);
+  return sizeof(float) * (size_t)s->B * s->Hq * decode_nchunk(s->B, s->Hkv, s->L) * (2 + (size_t)s->d);
 }
 
 static bool decode_cache_ok(const thrift_decode_cache* c) {
@@ -289,8 +289,10 @@ thrift_status thrift_decode_step(const thrift_decode_shape* shape, const void* q
 }
 
 thrift_status thrift_device_status(void* stream, uint32_t* detail) {
-  uint32_t w = 0;
+  uint32_t w = 0, wd = 0;
   if (read_and_clear_device_error(static_cast<cudaStream_t>(stream), &w) != cudaSuccess) return THRIFT_ERR_CUDA;
+  if (read_and_clear_decode_error(&wd) != cudaSuccess) return THRIFT_ERR_CUDA;
+  w |= wd << 8;
   if (detail != nullptr) *detail = w;
   return w != 0 ? THRIFT_ERR_TIMEOUT : THRIFT_OK;
 }

@@ -66,6 +66,12 @@ constexpr int kMaxW = 128;                          // mask words per query tile
 // Element pairs (bit t of 16, for pair t mod 16 of a row) whose exponential runs on the
 // FMA pipe; the rest run on the MUFU.
 constexpr uint32_t kPolyPairs = THRIFT_POLY_PAIRS;
+#ifndef THRIFT_MAX_PUBLISH_CHUNK
+#define THRIFT_MAX_PUBLISH_CHUNK 0
+#endif
+// How many of a tile's four 32-column exponential chunks a softmax warp finishes before it
+// hands the tile's running maximum to the next group (0: right after computing it).
+constexpr int kMaxPublishChunk = THRIFT_MAX_PUBLISH_CHUNK;
 
 // Operand rings: FP4 tiles use NLO slots of K (e2m1 + scales) and of V^T (e4m3);
 // BF16 tiles use NHI slots of bf16 K and V^T.  Producer and MMA issuer walk the
@@ -91,6 +97,18 @@ enum Bar : int {
 };
 
 __host__ __device__ constexpr int al(int x, int a) { return (x + a - 1) / a * a; }
+
+// Ring slot and use count of the n-th FP4 (NLO slots) or BF16 (NHI slots) tile, with
+// constant divisors in each branch.
+__device__ __forceinline__ void ring_pos(bool hi, int n, int& slot, int& use) {
+  if (hi) {
+    slot = n % NHI;
+    use = n / NHI;
+  } else {
+    slot = n % NLO;
+    use = n / NLO;
+  }
+}
 
 template <int D>
 struct Layout {
@@ -219,7 +237,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       int nlo = 0, nhi = 0;
       for (int j = 0; j < nj; ++j) {
         const bool hi = is_hi(j);
-        const int n = hi ? nhi : nlo, slots = hi ? NHI : NLO, slot = n % slots, use = n / slots;
+        int slot, use;
+        ring_pos(hi, hi ? nhi : nlo, slot, use);
         const int FULL = kside ? (hi ? KH_FULL : KL_FULL) : (hi ? VH_FULL : VL_FULL);
         const int EMPTY = kside ? (hi ? KH_EMPTY : KL_EMPTY) : (hi ? VH_EMPTY : VL_EMPTY);
         if (use > 0 && !mbar_wait(BAR(EMPTY + slot), (use - 1) & 1, abort, kWaitLimitNs)) {
@@ -279,7 +298,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!pv_wait(j - 2)) { ok = false; break; }
           }
         }
-        const int n = hi ? n_hi : n_lo, slots = hi ? NHI : NLO, slot = n % slots, use = n / slots;
+        int slot, use;
+        ring_pos(hi, hi ? n_hi : n_lo, slot, use);
         if (!mbar_wait(BAR((hi ? KH_FULL : KL_FULL) + slot), use & 1, abort, kWaitLimitNs)) { ok = false; break; }
         tc_fence_after();
         const uint32_t d_s = tmem + L::S_COL0 + 128 * s;
@@ -328,7 +348,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         if ((t & 31) == 0) mw = mrow[t >> 5];
         const bool hi = (mw >> (t & 31)) & 1u;
         const int s = t & 1, g = t % kGroups, u = t / kGroups;
-        const int n = hi ? n_hi : n_lo, slots = hi ? NHI : NLO, slot = n % slots, use = n / slots;
+        int slot, use;
+        ring_pos(hi, hi ? n_hi : n_lo, slot, use);
         if (!mbar_wait(BAR(P_FULL + kPRing * g + (u % kPRing)), (u / kPRing) & 1, abort, kWaitLimitNs) ||
             !mbar_wait(BAR((hi ? VH_FULL : VL_FULL) + slot), use & 1, abort, kWaitLimitNs)) {
           ok = false;
@@ -441,7 +462,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float m_new = fmaxf(m_prev, mloc * sc);
       mbuf[wg * 128 + r] = m_new;
       __syncwarp();
-      if (j + 1 < nj && lane == 0) mbar_arrive(mx_out);
+      if (kMaxPublishChunk == 0 && j + 1 < nj && lane == 0) mbar_arrive(mx_out);
       const float alpha = (m_prev == -INFINITY) ? 0.0f : ex2_approx(m_prev - m_new);  // O rescale
       const float beta = (m_ref == -INFINITY) ? 0.0f : ex2_approx(m_ref - m_new);     // own partial sum
       const uint64_t sc2 = f2pack(sc, sc);
@@ -462,6 +483,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       // run on the FMA pipe (polynomial), the others on the MUFU.
 #pragma unroll
       for (int ch = 0; ch < 4; ++ch) {
+        // hand m_j to the next group once this warp's exponentials are far enough along that
+        // the next group's (on the same sub-partition's MUFU) follow rather than overlap them
+        if (kMaxPublishChunk > 0 && ch == kMaxPublishChunk && j + 1 < nj) {
+          __syncwarp();
+          if (lane == 0) mbar_arrive(mx_out);
+        }
 #pragma unroll
         for (int t = 16 * ch; t < 16 * ch + 16; ++t) {
           const uint64_t y2 = ffma2(f2pack(__uint_as_float(v[2 * t]), __uint_as_float(v[2 * t + 1])), sc2, nb2);
@@ -497,6 +524,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_st8(p_base + 32 * (j % 3) + 8 * ch, pe);
         }
       }
+      if (kMaxPublishChunk >= 4 && j + 1 < nj) {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(mx_out);
+      }
       float r0, r1, r2, r3, r4, r5, r6, r7;
       f2unpack(acc[0], r0, r1);
       f2unpack(acc[1], r2, r3);
@@ -513,21 +544,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_fence_after();
         const uint64_t al2 = f2pack(alpha, alpha);
+        // the whole O row in one TMEM round trip: v (P is stored) holds it
+        const uint32_t o_addr = tmem + lane_base + L::O_COL;
 #pragma unroll
-        for (int c4 = 0; c4 < D / 32; ++c4) {
-          uint32_t ov[32];
-          const uint32_t o_addr = tmem + lane_base + L::O_COL + 32 * c4;
-          tmem_ld32(o_addr, ov);
-          tmem_ld_wait();
+        for (int c4 = 0; c4 < D / 32; ++c4) tmem_ld32(o_addr + 32 * c4, *reinterpret_cast<uint32_t(*)[32]>(&v[32 * c4]));
+        tmem_ld_wait();
 #pragma unroll
-          for (int c = 0; c < 32; c += 2) {
-            float a0, a1;
-            f2unpack(fmul2(f2pack(__uint_as_float(ov[c]), __uint_as_float(ov[c + 1])), al2), a0, a1);
-            ov[c] = __float_as_uint(a0);
-            ov[c + 1] = __float_as_uint(a1);
-          }
-          tmem_st32(o_addr, ov);
+        for (int c = 0; c < D; c += 2) {
+          float a0, a1;
+          f2unpack(fmul2(f2pack(__uint_as_float(v[c]), __uint_as_float(v[c + 1])), al2), a0, a1);
+          v[c] = __float_as_uint(a0);
+          v[c + 1] = __float_as_uint(a1);
         }
+#pragma unroll
+        for (int c4 = 0; c4 < D / 32; ++c4) tmem_st32(o_addr + 32 * c4, *reinterpret_cast<const uint32_t(*)[32]>(&v[32 * c4]));
       }
       tmem_st_wait();
       tc_fence_before();

@@ -94,19 +94,63 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
   return t;
 }
+__device__ __forceinline__ uint32_t globaltimer_lo() {
+  uint32_t t;
+  asm volatile("mov.u32 %0, %%globaltimer_lo;" : "=r"(t));
+  return t;
+}
+
+// try_wait with a suspend-time hint: a thread whose phase is not complete yet may be
+// suspended for up to `hint_ns` nanoseconds and is woken when the phase completes, so a
+// waiting warp stops issuing instructions instead of polling.
+__device__ __forceinline__ bool mbar_try_wait_suspend(uint32_t bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok) : "r"(bar), "r"(parity), "r"(hint_ns) : "memory");
+  return ok != 0;
+}
+
+// 0: poll with plain try_wait (measured faster in the attention kernel than sleeping
+// with a suspend-time hint, whose wake-up adds latency to every hand-off)
+#ifndef THRIFT_WAIT_HINT_NS
+#define THRIFT_WAIT_HINT_NS 0
+#endif
 
 // Bounded wait on an mbarrier phase.  Returns false (and never hangs) when
-// the wait exceeds `limit_ns` or when another role raised `*abort`.
+// the wait exceeds `limit_ns` or when another role raised `*abort` (both are
+// checked every 64 polls).
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort,
                                           uint64_t limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
-  uint64_t t0 = globaltimer_ns();
+  // the low 32 bits of the nanosecond timer: differences stay exact for limits below 4.29 s
+  const uint32_t t0 = globaltimer_lo();
   for (uint32_t it = 1;; ++it) {
+#if THRIFT_WAIT_HINT_NS > 0
+    if (mbar_try_wait_suspend(bar, parity, THRIFT_WAIT_HINT_NS)) return true;
+#else
     if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 255u) == 0u) {
+#endif
+    if ((it & 63u) == 0u) {
       if (*abort) return false;
-      if (globaltimer_ns() - t0 > limit_ns) return false;
+      if ((uint64_t)(globaltimer_lo() - t0) > limit_ns) return false;
     }
+  }
+}
+
+// mbar_wait for a thread that is not on the critical path (a producer running ahead):
+// it sleeps in try_wait between checks instead of polling, leaving its issue slots to
+// the other warps of its sub-partition.
+__device__ __forceinline__ bool mbar_wait_sleep(uint32_t bar, uint32_t parity, volatile int* abort,
+                                                uint64_t limit_ns) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint32_t t0 = globaltimer_lo();
+  for (;;) {
+    if (mbar_try_wait_suspend(bar, parity, 20000u)) return true;
+    if (*abort) return false;
+    if ((uint64_t)(globaltimer_lo() - t0) > limit_ns) return false;
   }
 }
 
@@ -195,6 +239,12 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint3
   d |= (uint64_t)1 << 46;
   d |= (uint64_t)(swz & 7u) << 61;
   return d;
+}
+
+// The descriptor of start address 0: add (address >> 4) for a tile (addresses below 256 KB).
+__host__ __device__ constexpr uint64_t smem_desc_tmpl(uint32_t lbo, uint32_t sbo, uint32_t swz) {
+  return (uint64_t)((lbo >> 4) & 0x3FFFu) << 16 | (uint64_t)((sbo >> 4) & 0x3FFFu) << 32 | (uint64_t)1 << 46 |
+         (uint64_t)(swz & 7u) << 61;
 }
 
 // Instruction descriptors (M = 128, FP32 accumulate, both operands K-major).

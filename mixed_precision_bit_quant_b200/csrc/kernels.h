@@ -57,10 +57,12 @@ struct DecodeArgs {
   float* lse;
   float* ws;  // [B*Hq][nchunk][2 + d] chunk softmax states
 };
-int decode_nchunk(int L);
-int decode_max_group();
+int decode_nchunk(int B, int Hkv, int L);  // splits per (b, kv head)
+bool decode_group_supported(int G);  // query heads per kv head: 1, 2, 4, 8 or 16
 cudaError_t launch_decode_quantize(const DecodeArgs& a, int t0, int t1, cudaStream_t s);
 cudaError_t launch_decode_step(const DecodeArgs& a, cudaStream_t s);
+// reads and clears the decode kernels' device error word (1: a chunk copy's wait gave up)
+cudaError_t read_and_clear_decode_error(uint32_t* word);
 
 cudaError_t read_and_clear_device_error(cudaStream_t s, uint32_t* word);
 

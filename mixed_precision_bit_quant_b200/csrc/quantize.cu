@@ -127,32 +127,12 @@ __global__ void __launch_bounds__(256) nvfp4_pack_kernel(
     const float den = __fmul_rn(sd, g);
     uint32_t lo = 0, hi = 0;
     if (sd > 0.0f) {
-      // The quotient x / den, correctly rounded, decides the code.  x * fl(1/den) is
-      // within 2 ulps of it; every e2m1 rounding threshold (0.25, 0.75, 1.25, 1.75,
-      // 2.5, 3.5, 5) has at most two significant bits, i.e. 21 zero low mantissa bits,
-      // so a product farther than 3 ulps from every such value rounds to the code of
-      // the exact quotient.  The few products that are that close (and no zero) take
-      // the correctly rounded division instead.
-      const float rcp = __frcp_rn(den);
-      float qv[16];
-      bool near = false;
 #pragma unroll
-      for (int e = 0; e < 16; ++e) {
-        qv[e] = __fmul_rn(f[e], rcp);
-        const uint32_t m = __float_as_uint(qv[e]) & 0x7FFFFFFFu;
-        near |= (m != 0u) && (((m + 3u) & 0x1FFFFFu) < 7u);
-      }
-      if (near) {
+      for (int e = 0; e < 4; ++e)
+        lo |= cvt_e2m1x2(__fdiv_rn(f[2 * e], den), __fdiv_rn(f[2 * e + 1], den)) << (8 * e);
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const uint32_t m = __float_as_uint(qv[e]) & 0x7FFFFFFFu;
-          if ((m != 0u) && (((m + 3u) & 0x1FFFFFu) < 7u)) qv[e] = __fdiv_rn(f[e], den);
-        }
-      }
-#pragma unroll
-      for (int e = 0; e < 4; ++e) lo |= cvt_e2m1x2(qv[2 * e], qv[2 * e + 1]) << (8 * e);
-#pragma unroll
-      for (int e = 0; e < 4; ++e) hi |= cvt_e2m1x2(qv[8 + 2 * e], qv[9 + 2 * e]) << (8 * e);
+      for (int e = 0; e < 4; ++e)
+        hi |= cvt_e2m1x2(__fdiv_rn(f[8 + 2 * e], den), __fdiv_rn(f[9 + 2 * e], den)) << (8 * e);
     }
     out[2 * b] = lo;
     out[2 * b + 1] = hi;
