@@ -189,14 +189,26 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint32_t* mrow = reinterpret_cast<uint32_t*>(smem + L::OFF_MASK);
   float* vsc = reinterpret_cast<float*>(smem + L::OFF_VSC);
 
-  if (tid == 0) {
-    for (int k = 0; k < NBAR; ++k) {
+  if (warp == 0) {
+    // the lanes of warp 0 initialise the barriers (Q_FULL is the K producer's, below)
+    for (int k = lane; k < NBAR; k += 32) {
       const bool by_group = (k >= S_FREE && k < S_FREE + 2) || (k >= P_FULL && k < P_FULL + kPRing * kGroups);
-      mbar_init(BAR(k), by_group ? 4 : 1);  // softmax barriers: one arrival per warp of the group
+      if (k != Q_FULL) mbar_init(BAR(k), by_group ? 4 : 1);  // softmax barriers: one arrival per warp of the group
     }
-    *abort = 0;
-    *reinterpret_cast<volatile uint32_t*>(smem + L::OFF_MISC + 8) = 0u;
+    if (lane == 0) {
+      *abort = 0;
+      *reinterpret_cast<volatile uint32_t*>(smem + L::OFF_MISC + 8) = 0u;
+    }
     fence_mbar_init();
+  } else if (warp == 4 * kGroups && lane == 0) {
+    // Q is loaded before the CTA-wide setup completes: its latency overlaps the rest
+    mbar_init(BAR(Q_FULL), 1);
+    fence_mbar_init();
+    mbar_expect_tx(BAR(Q_FULL), L::QFP4 + L::QBF + L::SF);
+    tma_load_3d(sb + L::OFF_QFP4, &tm_qfp4, 0, i * 128, bhq, BAR(Q_FULL));
+    tma_load_3d(sb + L::OFF_QBF, &tm_qbf, 0, i * 128, bhq, BAR(Q_FULL));
+    if (D == 128) tma_load_3d(sb + L::OFF_QBF + 16384, &tm_qbf, 64, i * 128, bhq, BAR(Q_FULL));
+    bulk_load(sb + L::OFF_QSF, p.q_sf_mma + ((size_t)bhq * p.T + i) * L::SF, L::SF, BAR(Q_FULL));
   }
   if (warp == 4 * kGroups + 1) {
     tmem_alloc(smem_u32(tmem_holder), 512);
@@ -225,12 +237,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // ahead of the softmax, bounded only by the QK^T that frees their stage.
       const bool kside = (warp == 4 * kGroups);
       if (kside) {
-        prefetch_tmap(&tm_qfp4); prefetch_tmap(&tm_kfp4); prefetch_tmap(&tm_qbf); prefetch_tmap(&tm_kbf);
-        mbar_expect_tx(BAR(Q_FULL), L::QFP4 + L::QBF + L::SF);
-        tma_load_3d(sb + L::OFF_QFP4, &tm_qfp4, 0, i * 128, bhq, BAR(Q_FULL));
-        tma_load_3d(sb + L::OFF_QBF, &tm_qbf, 0, i * 128, bhq, BAR(Q_FULL));
-        if (D == 128) tma_load_3d(sb + L::OFF_QBF + 16384, &tm_qbf, 64, i * 128, bhq, BAR(Q_FULL));
-        bulk_load(sb + L::OFF_QSF, p.q_sf_mma + ((size_t)bhq * p.T + i) * L::SF, L::SF, BAR(Q_FULL));
+        prefetch_tmap(&tm_kfp4); prefetch_tmap(&tm_kbf);
       } else {
         prefetch_tmap(&tm_vfp8); prefetch_tmap(&tm_vbf);
       }
