@@ -256,7 +256,10 @@ THRIFT_API thrift_status thrift_attn_fwd_mx(const thrift_shape *shape, const thr
  * with ties to the even code and saturated, sign kept; tokens [0, 128) (the
  * sink tile) and [L - 128, L) (the local window) are read from the BF16 cache,
  * every other token from its quantised form; the query stays BF16; logits
- * q . k * scale, exact softmax over all L tokens in FP32, no rounding of P.
+ * q . k * scale, exact softmax over all L tokens in FP32.  Both products run on
+ * the tensor cores with TF32 operands: the e2m1, e4m3 and BF16 values are exact
+ * in TF32, and P (times V's power-of-two block scale) enters as the sum of two
+ * TF32 terms, carrying it to about 21 significant bits.
  * ------------------------------------------------------------------------ */
 typedef struct {
   int32_t B, Hq, Hkv, L, d; /* L: cached tokens (>= 1); d in {64, 128}; Hq / Hkv in {1, 2, 4, 8, 16} */
@@ -306,7 +309,8 @@ THRIFT_API thrift_status thrift_decode_step(const thrift_decode_shape *shape, co
  * words.  Returns THRIFT_ERR_TIMEOUT if a kernel's bounded wait gave up since
  * the last call (the kernel then returned early and its outputs are
  * undefined); *detail (if non-NULL) receives the raw error word: bits 0-2
- * from thrift_attn_fwd (1 producer, 2 tensor-core issuer, 4 softmax); the
+ * from thrift_attn_fwd (1 producer, 2 tensor-core issuer, 4 softmax), bit 8
+ * from thrift_decode_step (a CTA's wait for its bulk-copied cache codes); the
  * other kernels wait on nothing and set no bit.
  */
 THRIFT_API thrift_status thrift_device_status(void *stream, uint32_t *detail);

@@ -8,15 +8,17 @@
 // cache grows a token at a time), K as MXFP4 and V as MXFP8 (e4m3), one e8m0
 // scale per 32 channels of the token; tokens [0, 128) and [L - 128, L) are read
 // from the BF16 cache; the query stays BF16; exact softmax over all L tokens in
-// FP32 on CUDA cores (the step reads each cached byte once: HBM-bound).
+// FP32, the two products on the tensor cores with exact operands (the step reads
+// each cached byte once: HBM-bound).
 //
 // Kernels:
 //   decode_quantize_kernel  per-token MX quantisation of cache rows [t0, t1)
 //   decode_partial_kernel   one CTA per (b, kv head, chunk of 256 tokens), all G
-//                           query heads of the group: logits (one lane per token),
-//                           chunk max / exp sum per head, P.V (one lane per d/32
-//                           channels, one warp per token stream, four tokens'
-//                           rows loaded together); writes the
+//                           query heads of the group: logits S = K Q^T and
+//                           O = P V on the tensor cores (mma.sync, TF32 operands:
+//                           the e2m1, e4m3 and BF16 values are exact in TF32,
+//                           P enters as two TF32 terms), dequantisation in
+//                           registers, chunk max / exp sum per head; writes the
 //                           chunk's softmax state (max, sum, unnormalised O)
 //   decode_merge_kernel     combines the chunks' states per query head.
 #include "dev.cuh"
@@ -123,96 +125,255 @@ struct DecParams {
   float scale;
 };
 
-// Shared memory of one CTA for a group of G query heads (floats).
+constexpr int kPS = kChunk + 4;  // row stride of the probabilities in shared memory (spreads banks)
+
+// Shared memory of one CTA for a group of G query heads, in floats: the chunk's staged e2m1
+// K codes and e4m3 V codes, the group's query rows, the chunk's
+// logits / probabilities, the per-head maximum and sum, and every warp's partial P.V --
+// which reuses the K codes' space once the logits are done, when it fits there (G <= 4).
+__host__ __device__ constexpr int osum_floats(int D, int G) { return (kThreads / 32) * G * D; }
+__host__ __device__ constexpr int kstage_floats(int D) { return kChunk * (D / 2) / 4; }
+__host__ __device__ constexpr int vstage_floats(int D) { return kChunk * D / 4; }
+__host__ __device__ constexpr bool osum_in_kstage(int D, int G) { return osum_floats(D, G) <= kstage_floats(D); }
 __host__ __device__ constexpr int partial_smem_floats(int D, int G) {
-  return G * D + G * kChunk + 2 * G + (kThreads / 32) * G * D;
+  return kstage_floats(D) + vstage_floats(D) + G * D + G * kPS + 2 * G +
+         (osum_in_kstage(D, G) ? 0 : osum_floats(D, G)) + 4 /* mbarrier */;
 }
 
+__device__ uint32_t g_decode_error_word;
+constexpr uint64_t kStageWaitNs = 2000000000ull;  // 2 s: far above any legitimate copy
+
+// D[16x8] += A[16x8] B[8x8]: TF32 operands (the top 19 bits of FP32 registers), FP32
+// accumulation.  Fragments: a0 (row g, col t), a1 (row g+8, col t), a2 (row g, col t+4),
+// a3 (row g+8, col t+4); b0 (row t, col g), b1 (row t+4, col g); d0 (row g, col 2t),
+// d1 (row g, col 2t+1), d2 (row g+8, col 2t), d3 (row g+8, col 2t+1); g = lane / 4,
+// t = lane % 4.
+__device__ __forceinline__ void mma_tf32(float (&d)[4], float a0, float a1, float a2, float a3, float b0, float b1) {
+  asm("mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(__float_as_uint(a0)), "r"(__float_as_uint(a1)), "r"(__float_as_uint(a2)), "r"(__float_as_uint(a3)),
+        "r"(__float_as_uint(b0)), "r"(__float_as_uint(b1)));
+}
+
+// Channels 32c + 8t .. 32c + 8t + 7 of cache row `row` of K, as FP32: the BF16 row for a
+// high-precision token, else the e2m1 codes (bytes 16c + 4t .. +3 of the row) unscaled.
+template <int D>
+__device__ __forceinline__ void load_k8(const DecParams& p, long long row, bool valid, bool high, int c, int t,
+                                        float (&a)[8]) {
+  if (!valid) {
+#pragma unroll
+    for (int m = 0; m < 8; ++m) a[m] = 0.0f;
+  } else if (high) {
+    const uint4 u = __ldg(reinterpret_cast<const uint4*>(p.k + row * D + 32 * c + 8 * t));
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      a[2 * e] = __uint_as_float(w[e] << 16);
+      a[2 * e + 1] = __uint_as_float(w[e] & 0xFFFF0000u);
+    }
+  } else {
+    const uint32_t w = __ldg(reinterpret_cast<const uint32_t*>(p.kc + row * (D / 2) + 16 * c + 4 * t));
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float2 x = e2m1x2_to_float2((w >> (8 * j)) & 0xFFu);
+      a[2 * j] = x.x;
+      a[2 * j + 1] = x.y;
+    }
+  }
+}
+
+// Channels 32c + 4g .. 32c + 4g + 3 of cache row `row` of V, as FP32: the BF16 row for a
+// high-precision token, else the e4m3 codes unscaled.
+template <int D>
+__device__ __forceinline__ void load_v4(const DecParams& p, long long row, bool valid, bool high, int c, int g,
+                                        float (&x)[4]) {
+  if (!valid) {
+#pragma unroll
+    for (int m = 0; m < 4; ++m) x[m] = 0.0f;
+  } else if (high) {
+    const uint2 u = __ldg(reinterpret_cast<const uint2*>(p.v + row * D + 32 * c + 4 * g));
+    x[0] = __uint_as_float(u.x << 16);
+    x[1] = __uint_as_float(u.x & 0xFFFF0000u);
+    x[2] = __uint_as_float(u.y << 16);
+    x[3] = __uint_as_float(u.y & 0xFFFF0000u);
+  } else {
+    const uint32_t w = __ldg(reinterpret_cast<const uint32_t*>(p.vc + row * D + 32 * c + 4 * g));
+    const float2 lo = e4m3x2_to_float2(w & 0xFFFFu), hi = e4m3x2_to_float2(w >> 16);
+    x[0] = lo.x;
+    x[1] = lo.y;
+    x[2] = hi.x;
+    x[3] = hi.y;
+  }
+}
+
+// The e8m0 scale codes of one cache row (one byte per 32-channel block, block 0 lowest).
+template <int D>
+__device__ __forceinline__ uint32_t load_scales(const uint8_t* sc, long long row) {
+  constexpr int NB = D / 32;
+  if (NB == 4) return __ldg(reinterpret_cast<const uint32_t*>(sc + row * 4));
+  return (uint32_t)__ldg(reinterpret_cast<const uint16_t*>(sc + row * 2));
+}
+
+// FP32 -> two TF32 terms whose sum carries it to ~21 bits: hi keeps the top 11
+// significant bits, lo = x - hi (exact in FP32) is rounded by the tensor core.
+__device__ __forceinline__ void split_tf32(float x, float& hi, float& lo) {
+  hi = __uint_as_float(__float_as_uint(x) & 0xFFFFE000u);
+  lo = x - hi;
+}
+
+// Four CTAs per SM for groups of up to 4 heads (64 registers a thread), two above: with
+// the chunk's codes staged by bulk copies, more resident CTAs keep more of the cache in
+// flight.
 template <int D, int G>
-__global__ void __launch_bounds__(kThreads) decode_partial_kernel(const DecParams p) {
-  constexpr int CPL = D / 32;  // channels per lane in the P.V phase
-  constexpr int NB = D / 32;   // 32-channel scale blocks per row
+__global__ void __launch_bounds__(kThreads, G <= 4 ? 4 : 2) decode_partial_kernel(const DecParams p) {
+  constexpr int NB = D / 32;         // 32-channel scale blocks per row
+  constexpr int NT = (G + 7) / 8;    // 8-head column tiles of the products
   const int chunk = blockIdx.x, bk = blockIdx.y, b = bk / p.Hkv, hk = bk % p.Hkv;
-  const int t0 = chunk * kChunk, t1 = min(p.L, t0 + kChunk), nt = t1 - t0;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  extern __shared__ float dsm[];
-  float* qs = dsm;                 // [G][D]
-  float* ps = qs + G * D;          // [G][kChunk]
-  float* red = ps + G * kChunk;    // [G][2]
-  float* osum = red + 2 * G;       // [8 warps][G][D]
+  const int t0 = chunk * kChunk, nt = min(p.L, t0 + kChunk) - t0;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, tq = lane & 3;
+  extern __shared__ __align__(16) float dsm[];
+  uint8_t* kcs = reinterpret_cast<uint8_t*>(dsm);                 // [kChunk][D/2] staged K codes
+  uint8_t* vcs = kcs + kChunk * (D / 2);                           // [kChunk][D] staged V codes
+  float* qs = dsm + kstage_floats(D) + vstage_floats(D);           // [G][D]
+  float* ps = qs + G * D;                                          // [G][kPS]
+  float* red = ps + G * kPS;                                       // [G][2]
+  float* osum = osum_in_kstage(D, G) ? dsm : red + 2 * G;          // [8 warps][G][D]
+  uint64_t* stage_bar = reinterpret_cast<uint64_t*>(red + 2 * G + (osum_in_kstage(D, G) ? 0 : osum_floats(D, G)));
+  const long long row0 = (long long)bk * p.L + t0;  // cache row of the chunk's first token
+  // A whole chunk's codes are contiguous in the cache: one bulk copy each for K and V,
+  // issued first so that the CTA's bytes are all in flight while it sets up.
+  const bool staged = (nt == kChunk);
+  const uint32_t bar = smem_u32(stage_bar);
+  if (staged && threadIdx.x == 0) {
+    mbar_init(bar, 1);
+    fence_mbar_init();
+    mbar_expect_tx(bar, kChunk * (D / 2) + kChunk * D);
+    bulk_load(smem_u32(kcs), p.kc + row0 * (D / 2), kChunk * (D / 2), bar);
+    bulk_load(smem_u32(vcs), p.vc + row0 * D, kChunk * D, bar);
+  }
   for (int i = threadIdx.x; i < G * D; i += kThreads)
     qs[i] = __bfloat162float(p.q[((long long)b * p.Hq + hk * G + i / D) * D + i % D]);
   __syncthreads();
-  const long long row0 = (long long)bk * p.L;
-  // ---- logits: one thread per token, all G heads, channels ascending; the whole
-  // row is loaded before it is used, so each thread has its row's bytes in flight
-  for (int tt = threadIdx.x; tt < nt; tt += kThreads) {
+  auto high = [&](int tt) -> bool {
     const int t = t0 + tt;
-    const long long row = row0 + t;
-    float s[G];
+    return t < kSink || t >= p.L - kWindow;
+  };
+
+  // A warp whose 32 tokens are all quantised, in a staged chunk, takes the fast path: its
+  // codes come from the staged copy and its scale words (lane l: token 32w + l) from one
+  // load per lane, passed between lanes by shuffles.  Warps that meet the sink, the window
+  // or a partial last chunk load per element from global memory as they go.
+  const int wt0 = 32 * warp;
+  const bool fast = staged && (t0 + wt0 >= kSink) && (t0 + wt0 + 32 <= p.L - kWindow);
+  uint32_t ksw = 0u, vsw = 0u;
+  if (fast) {
+    ksw = load_scales<D>(p.ksc, row0 + wt0 + lane);
+    vsw = load_scales<D>(p.vsc, row0 + wt0 + lane);
+  }
+  if (staged) {
+    // every thread sees the copy complete (bounded: on a timeout the error word is set and
+    // the CTA waits once more, again bounded, for its own copies before it returns)
+    volatile int no_abort = 0;
+    const bool landed = mbar_wait(bar, 0, &no_abort, kStageWaitNs);
+    if (!__syncthreads_and(landed)) {
+      if (threadIdx.x == 0) {
+        atomicOr(&g_decode_error_word, 1u);
+        mbar_wait(bar, 0, &no_abort, kStageWaitNs);
+      }
+      __syncthreads();
+      return;
+    }
+  }
+
+  // ---- logits S = K Q^T on the tensor cores (mma.sync TF32: e2m1, BF16 and the BF16
+  // query are exact in TF32, so every product is exact and the sums are FP32).  Warp w
+  // takes the chunk's tokens [32w, 32w + 32) as two 16-row tiles; the 8 columns are
+  // query heads.  Within 32-channel block c, MMA step j pairs k = t with channel
+  // 32c + 8t + 2j and k = t + 4 with the next channel, so that a thread's four codes of
+  // a row are one 32-bit word.  Each block's product is scaled by its row's e8m0 scale
+  // (a power of two: exact) before it joins the row's sum.
+  {
+    float bq[NT][NB][8];
 #pragma unroll
-    for (int h = 0; h < G; ++h) s[h] = 0.0f;
-    if (t < kSink || t >= p.L - kWindow) {
-      const uint4* kr = reinterpret_cast<const uint4*>(p.k + row * D);
-      uint4 u[D / 8];
+    for (int n = 0; n < NT; ++n)
 #pragma unroll
-      for (int c8 = 0; c8 < D / 8; ++c8) u[c8] = __ldg(kr + c8);
+      for (int c = 0; c < NB; ++c)
 #pragma unroll
-      for (int c8 = 0; c8 < D / 8; ++c8) {
-        const uint32_t w[4] = {u[c8].x, u[c8].y, u[c8].z, u[c8].w};
+        for (int m = 0; m < 8; ++m) bq[n][c][m] = (8 * n + g < G) ? qs[(8 * n + g) * D + 32 * c + 8 * tq + m] : 0.0f;
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float x0 = __uint_as_float(w[e] << 16), x1 = __uint_as_float(w[e] & 0xFFFF0000u);
-          const int c = 8 * c8 + 2 * e;
+    for (int tile = 0; tile < 2; ++tile) {
+      const int r_lo = wt0 + 16 * tile + g, r_hi = r_lo + 8;
+      const bool v_lo = r_lo < nt, v_hi = r_hi < nt;
+      const bool h_lo = v_lo && high(r_lo), h_hi = v_hi && high(r_hi);
+      uint32_t ks_lo = 0x7F7F7F7Fu, ks_hi = 0x7F7F7F7Fu;
+      if (fast) {
+        ks_lo = __shfl_sync(0xffffffffu, ksw, 16 * tile + g);
+        ks_hi = __shfl_sync(0xffffffffu, ksw, 16 * tile + g + 8);
+      } else {
+        if (v_lo && !h_lo) ks_lo = load_scales<D>(p.ksc, row0 + r_lo);
+        if (v_hi && !h_hi) ks_hi = load_scales<D>(p.ksc, row0 + r_hi);
+      }
+      float s[NT][4];
 #pragma unroll
-          for (int h = 0; h < G; ++h) s[h] = fmaf(qs[h * D + c + 1], x1, fmaf(qs[h * D + c], x0, s[h]));
+      for (int n = 0; n < NT; ++n)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) s[n][e] = 0.0f;
+#pragma unroll
+      for (int c = 0; c < NB; ++c) {
+        float a_lo[8], a_hi[8];
+        if (fast) {
+          const uint32_t kw_lo = *reinterpret_cast<const uint32_t*>(kcs + r_lo * (D / 2) + 16 * c + 4 * tq);
+          const uint32_t kw_hi = *reinterpret_cast<const uint32_t*>(kcs + r_hi * (D / 2) + 16 * c + 4 * tq);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const float2 xl = e2m1x2_to_float2((kw_lo >> (8 * j)) & 0xFFu);
+            const float2 xh = e2m1x2_to_float2((kw_hi >> (8 * j)) & 0xFFu);
+            a_lo[2 * j] = xl.x;
+            a_lo[2 * j + 1] = xl.y;
+            a_hi[2 * j] = xh.x;
+            a_hi[2 * j + 1] = xh.y;
+          }
+        } else {
+          load_k8<D>(p, row0 + r_lo, v_lo, h_lo, c, tq, a_lo);
+          load_k8<D>(p, row0 + r_hi, v_hi, h_hi, c, tq, a_hi);
+        }
+        const float sc_lo = e8m0_value((ks_lo >> (8 * c)) & 0xFFu), sc_hi = e8m0_value((ks_hi >> (8 * c)) & 0xFFu);
+#pragma unroll
+        for (int n = 0; n < NT; ++n) {
+          float cb[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            mma_tf32(cb, a_lo[2 * j], a_hi[2 * j], a_lo[2 * j + 1], a_hi[2 * j + 1], bq[n][c][2 * j],
+                     bq[n][c][2 * j + 1]);
+          s[n][0] = fmaf(cb[0], sc_lo, s[n][0]);
+          s[n][1] = fmaf(cb[1], sc_lo, s[n][1]);
+          s[n][2] = fmaf(cb[2], sc_hi, s[n][2]);
+          s[n][3] = fmaf(cb[3], sc_hi, s[n][3]);
         }
       }
-    } else {
-      const uint4* kr = reinterpret_cast<const uint4*>(p.kc + row * (D / 2));
-      uint4 u[NB];
-      uint32_t scw[NB];
 #pragma unroll
-      for (int c32 = 0; c32 < NB; ++c32) {
-        u[c32] = __ldg(kr + c32);
-        scw[c32] = __ldg(p.ksc + row * NB + c32);
-      }
+      for (int n = 0; n < NT; ++n)
 #pragma unroll
-      for (int c32 = 0; c32 < NB; ++c32) {
-        const float sc = e8m0_value(scw[c32]);
-        const uint32_t w[4] = {u[c32].x, u[c32].y, u[c32].z, u[c32].w};
-        float blk[G];
-#pragma unroll
-        for (int h = 0; h < G; ++h) blk[h] = 0.0f;
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-#pragma unroll
-          for (int n = 0; n < 4; ++n) {
-            const float2 x = e2m1x2_to_float2((w[e] >> (8 * n)) & 0xFFu);
-            const int c = 32 * c32 + 8 * e + 2 * n;
-#pragma unroll
-            for (int h = 0; h < G; ++h) blk[h] = fmaf(qs[h * D + c + 1], x.y, fmaf(qs[h * D + c], x.x, blk[h]));
+        for (int e = 0; e < 2; ++e) {
+          const int h = 8 * n + 2 * tq + e;
+          if (h < G) {
+            if (v_lo) ps[h * kPS + r_lo] = s[n][e] * p.scale;
+            if (v_hi) ps[h * kPS + r_hi] = s[n][2 + e] * p.scale;
           }
         }
-        // the block's scale is a power of two: scaling the block's partial sum is exact
-#pragma unroll
-        for (int h = 0; h < G; ++h) s[h] = fmaf(blk[h], sc, s[h]);
-      }
     }
-#pragma unroll
-    for (int h = 0; h < G; ++h) ps[h * kChunk + tt] = s[h] * p.scale;
   }
   __syncthreads();
   // ---- chunk maximum and exponential sum per head (one warp per head)
   for (int h = warp; h < G; h += kThreads / 32) {
     float m = -INFINITY;
-    for (int i = lane; i < nt; i += 32) m = fmaxf(m, ps[h * kChunk + i]);
+    for (int i = lane; i < nt; i += 32) m = fmaxf(m, ps[h * kPS + i]);
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
     float l = 0.0f;
     for (int i = lane; i < nt; i += 32) {
-      const float e = __expf(ps[h * kChunk + i] - m);
-      ps[h * kChunk + i] = e;
+      const float e = __expf(ps[h * kPS + i] - m);
+      ps[h * kPS + i] = e;
       l += e;
     }
 #pragma unroll
@@ -223,80 +384,85 @@ __global__ void __launch_bounds__(kThreads) decode_partial_kernel(const DecParam
     }
   }
   __syncthreads();
-  // ---- P.V: warp w takes tokens t0 + w, t0 + w + 8, ... four at a time (their rows
-  // loaded together); lane owns CPL consecutive channels
-  float acc[G][CPL];
+  // ---- P.V on the tensor cores: O^T[channel][head] += V^T[channel][token] P^T[token][head]
+  // over the warp's 32 tokens, 8 per step (k = t: token base + t, k = t + 4: token
+  // base + t + 4).  Tile (c, u) of block c: row g is channel 32c + 4g + 2u and row g+8 the
+  // next, so that a thread's channels of a token are four consecutive bytes.  V's e8m0
+  // scale (per token and block) goes into P (exact powers of two), and P enters as two
+  // TF32 terms.
+  float acc[NT][NB][2][4];
 #pragma unroll
-  for (int h = 0; h < G; ++h)
+  for (int n = 0; n < NT; ++n)
 #pragma unroll
-    for (int c = 0; c < CPL; ++c) acc[h][c] = 0.0f;
-  const int c0 = lane * CPL;
-  constexpr int U = 4;
-  for (int tb = warp; tb < nt; tb += U * (kThreads / 32)) {
-    // raw row bytes of U tokens first: BF16 rows 2*CPL bytes (w0: channels c0, c0+1;
-    // w1: c0+2, c0+3), FP8 rows CPL bytes (w0)
-    uint32_t w0[U], w1[U];
-    float sc[U];
-    bool hp[U];
+    for (int c = 0; c < NB; ++c)
 #pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const int tt = tb + u * (kThreads / 32);
-      const int t = t0 + tt;
-      const long long row = row0 + t;
-      hp[u] = t < kSink || t >= p.L - kWindow;
-      w0[u] = 0u;
-      w1[u] = 0u;
-      sc[u] = 0.0f;
-      if (tt < nt) {
-        if (hp[u]) {
-          if (CPL == 4) {
-            const uint2 x = __ldg(reinterpret_cast<const uint2*>(p.v + row * D + c0));
-            w0[u] = x.x;
-            w1[u] = x.y;
-          } else {
-            w0[u] = __ldg(reinterpret_cast<const uint32_t*>(p.v + row * D + c0));
-          }
-        } else {
-          w0[u] = CPL == 4 ? __ldg(reinterpret_cast<const uint32_t*>(p.vc + row * D + c0))
-                           : (uint32_t)__ldg(reinterpret_cast<const uint16_t*>(p.vc + row * D + c0));
-          sc[u] = e8m0_value(__ldg(p.vsc + row * NB + c0 / 32));
-        }
-      }
+      for (int u = 0; u < 2; ++u)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc[n][c][u][e] = 0.0f;
+#pragma unroll
+  for (int step = 0; step < 4; ++step) {
+    const int ta = wt0 + 8 * step + tq, tb = ta + 4;
+    const bool va = ta < nt, vb = tb < nt;
+    const bool ha = va && high(ta), hb = vb && high(tb);
+    uint32_t vs_a = 0x7F7F7F7Fu, vs_b = 0x7F7F7F7Fu;
+    if (fast) {
+      vs_a = __shfl_sync(0xffffffffu, vsw, 8 * step + tq);
+      vs_b = __shfl_sync(0xffffffffu, vsw, 8 * step + tq + 4);
+    } else {
+      if (va && !ha) vs_a = load_scales<D>(p.vsc, row0 + ta);
+      if (vb && !hb) vs_b = load_scales<D>(p.vsc, row0 + tb);
+    }
+    float pa[NT], pb[NT];
+#pragma unroll
+    for (int n = 0; n < NT; ++n) {
+      const int h = 8 * n + g;
+      pa[n] = (h < G && va) ? ps[h * kPS + ta] : 0.0f;
+      pb[n] = (h < G && vb) ? ps[h * kPS + tb] : 0.0f;
     }
 #pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const int tt = tb + u * (kThreads / 32);
-      if (tt >= nt) break;
-      float x[CPL];
-      if (hp[u]) {
-        x[0] = __uint_as_float(w0[u] << 16);
-        x[1] = __uint_as_float(w0[u] & 0xFFFF0000u);
-        if (CPL == 4) {
-          x[2 % CPL] = __uint_as_float(w1[u] << 16);
-          x[3 % CPL] = __uint_as_float(w1[u] & 0xFFFF0000u);
-        }
+    for (int c = 0; c < NB; ++c) {
+      float xa[4], xb[4];
+      if (fast) {
+        const uint32_t wa = *reinterpret_cast<const uint32_t*>(vcs + ta * D + 32 * c + 4 * g);
+        const uint32_t wb = *reinterpret_cast<const uint32_t*>(vcs + tb * D + 32 * c + 4 * g);
+        const float2 a0 = e4m3x2_to_float2(wa & 0xFFFFu), a1 = e4m3x2_to_float2(wa >> 16);
+        const float2 b0 = e4m3x2_to_float2(wb & 0xFFFFu), b1 = e4m3x2_to_float2(wb >> 16);
+        xa[0] = a0.x; xa[1] = a0.y; xa[2] = a1.x; xa[3] = a1.y;
+        xb[0] = b0.x; xb[1] = b0.y; xb[2] = b1.x; xb[3] = b1.y;
       } else {
-        const float2 a = e4m3x2_to_float2(w0[u] & 0xFFFFu);
-        x[0] = a.x * sc[u];
-        x[1] = a.y * sc[u];
-        if (CPL == 4) {
-          const float2 bq = e4m3x2_to_float2(w0[u] >> 16);
-          x[2 % CPL] = bq.x * sc[u];
-          x[3 % CPL] = bq.y * sc[u];
-        }
+        load_v4<D>(p, row0 + ta, va, ha, c, g, xa);
+        load_v4<D>(p, row0 + tb, vb, hb, c, g, xb);
       }
+      const float sa = e8m0_value((vs_a >> (8 * c)) & 0xFFu), sb = e8m0_value((vs_b >> (8 * c)) & 0xFFu);
 #pragma unroll
-      for (int h = 0; h < G; ++h) {
-        const float pw = ps[h * kChunk + tt];
+      for (int n = 0; n < NT; ++n) {
+        float pa_hi, pa_lo, pb_hi, pb_lo;
+        split_tf32(pa[n] * sa, pa_hi, pa_lo);
+        split_tf32(pb[n] * sb, pb_hi, pb_lo);
 #pragma unroll
-        for (int c = 0; c < CPL; ++c) acc[h][c] = fmaf(pw, x[c], acc[h][c]);
+        for (int u = 0; u < 2; ++u) {
+          mma_tf32(acc[n][c][u], xa[2 * u], xa[2 * u + 1], xb[2 * u], xb[2 * u + 1], pa_hi, pb_hi);
+          mma_tf32(acc[n][c][u], xa[2 * u], xa[2 * u + 1], xb[2 * u], xb[2 * u + 1], pa_lo, pb_lo);
+        }
       }
     }
   }
 #pragma unroll
-  for (int h = 0; h < G; ++h)
+  for (int n = 0; n < NT; ++n)
 #pragma unroll
-    for (int c = 0; c < CPL; ++c) osum[(warp * G + h) * D + c0 + c] = acc[h][c];
+    for (int c = 0; c < NB; ++c)
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const int h = 8 * n + 2 * tq, ch = 32 * c + 4 * g + 2 * u;
+        if (h < G) {
+          osum[(warp * G + h) * D + ch] = acc[n][c][u][0];
+          osum[(warp * G + h) * D + ch + 1] = acc[n][c][u][2];
+        }
+        if (h + 1 < G) {
+          osum[(warp * G + h + 1) * D + ch] = acc[n][c][u][1];
+          osum[(warp * G + h + 1) * D + ch + 1] = acc[n][c][u][3];
+        }
+      }
   __syncthreads();
   // ---- chunk state: [max, sum, O[0..D)] per head
   float* st = p.ws + ((long long)bk * p.nchunk + chunk) * G * (2 + D);
@@ -342,11 +508,16 @@ int decode_nchunk(int B, int Hkv, int L) {
   return (L + dec::kChunk - 1) / dec::kChunk;
 }
 
-// The decode kernels wait on nothing, so they never set an error; the word exists so
-// that thrift_device_status reads the same interface for every kernel of the library.
+// Bit 0: a decode step's CTA gave up waiting for its staged cache bytes.
 cudaError_t read_and_clear_decode_error(uint32_t* word) {
-  *word = 0;
-  return cudaSuccess;
+  uint32_t w = 0;
+  cudaError_t e = cudaMemcpyFromSymbol(&w, dec::g_decode_error_word, sizeof(w));
+  if (e == cudaSuccess && w != 0) {
+    const uint32_t zero = 0;
+    e = cudaMemcpyToSymbol(dec::g_decode_error_word, &zero, sizeof(zero));
+  }
+  *word = w;
+  return e;
 }
 
 cudaError_t launch_decode_quantize(const DecodeArgs& a, int t0, int t1, cudaStream_t s) {

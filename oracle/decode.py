@@ -19,8 +19,8 @@ attention.  The page gives no formats or sizes, so this library fixes them:
 * the query of the step stays BF16 (decode is bound by reading the cache, so
   there is no low-bit query product to gain);
 * query head h reads kv head h // (Hq / Hkv); logits q . k_t / sqrt(d); exact
-  softmax over all L tokens (no P rounding: the products run on CUDA cores in
-  FP32); output sum_t p_t v_t and LSE = max + ln(sum).
+  softmax over all L tokens (P is not rounded); output sum_t p_t v_t and
+  LSE = max + ln(sum).
 
 Parity pins: tests/test_oracle_decode.py.
 """
