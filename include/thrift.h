@@ -257,9 +257,12 @@ THRIFT_API thrift_status thrift_attn_fwd_mx(const thrift_shape *shape, const thr
  * sink tile) and [L - 128, L) (the local window) are read from the BF16 cache,
  * every other token from its quantised form; the query stays BF16; logits
  * q . k * scale, exact softmax over all L tokens in FP32.  Both products run on
- * the tensor cores with TF32 operands: the e2m1, e4m3 and BF16 values are exact
- * in TF32, and P (times V's power-of-two block scale) enters as the sum of two
- * TF32 terms, carrying it to about 21 significant bits.
+ * the tensor cores.  Logits: FP16 operands for quantised tokens (the e2m1
+ * codes are exact; the query is scaled per head by a power of two that puts
+ * its largest component in [2^14, 2^15), so components more than 2^28 below it
+ * lose bits to FP16 subnormals)
+ * and TF32 for the BF16 rows; P.V: TF32, the e4m3 codes exact and P (times V's
+ * power-of-two block scale) as the sum of two TF32 terms, about 21 bits.
  * ------------------------------------------------------------------------ */
 typedef struct {
   int32_t B, Hq, Hkv, L, d; /* L: cached tokens (>= 1); d in {64, 128}; Hq / Hkv in {1, 2, 4, 8, 16} */

@@ -214,6 +214,24 @@ __device__ __forceinline__ uint32_t load_scales(const uint8_t* sc, long long row
   return (uint32_t)__ldg(reinterpret_cast<const uint16_t*>(sc + row * 2));
 }
 
+// D[16x8] += A[16x16] B[16x8]: FP16 operands, FP32 accumulation.  Fragments (two FP16
+// per register, the lower k in the low half): a0 (row g, k 2t..2t+1), a1 (row g+8,
+// k 2t..2t+1), a2 (row g, k 2t+8..2t+9), a3 (row g+8, k 2t+8..2t+9); b0 (k 2t..2t+1,
+// col g), b1 (k 2t+8..2t+9, col g); d as for mma_tf32.
+__device__ __forceinline__ void mma_f16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
+                                        uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Two e2m1 codes (one byte, element 2t in the low nibble) -> f16x2, exact.
+__device__ __forceinline__ uint32_t e2m1x2_to_h2(uint32_t byte) {
+  uint32_t r;
+  asm("{\n\t.reg .b8 t;\n\tmov.b16 {t, _}, %1;\n\tcvt.rn.f16x2.e2m1x2 %0, t;\n\t}" : "=r"(r) : "h"((unsigned short)byte));
+  return r;
+}
+
 // FP32 -> two TF32 terms whose sum carries it to ~21 bits: hi keeps the top 11
 // significant bits, lo = x - hi (exact in FP32) is rounded by the tensor core.
 __device__ __forceinline__ void split_tf32(float x, float& hi, float& lo) {
@@ -285,14 +303,93 @@ __global__ void __launch_bounds__(kThreads, G <= 4 ? 4 : 2) decode_partial_kerne
     }
   }
 
-  // ---- logits S = K Q^T on the tensor cores (mma.sync TF32: e2m1, BF16 and the BF16
-  // query are exact in TF32, so every product is exact and the sums are FP32).  Warp w
-  // takes the chunk's tokens [32w, 32w + 32) as two 16-row tiles; the 8 columns are
-  // query heads.  Within 32-channel block c, MMA step j pairs k = t with channel
-  // 32c + 8t + 2j and k = t + 4 with the next channel, so that a thread's four codes of
-  // a row are one 32-bit word.  Each block's product is scaled by its row's e8m0 scale
-  // (a power of two: exact) before it joins the row's sum.
-  {
+  // ---- logits S = K Q^T on the tensor cores.  Warp w takes the chunk's tokens
+  // [32w, 32w + 32) as two 16-row tiles; the 8 columns are query heads.  Each 32-channel
+  // block's product is scaled by its row's e8m0 scale (a power of two: exact) before it
+  // joins the row's sum.
+  //   Fast warps: mma.sync m16n8k16 FP16.  The e2m1 codes are exact in FP16 (one
+  // hardware e2m1x2 -> f16x2 conversion per byte), and the query enters as FP16 after a
+  // per-head power-of-two scaling 2^-e (e = floor(log2 amax) - 14) that puts its largest
+  // component in [2^14, 2^15); components more than 2^28 below it fall into FP16
+  // subnormals and lose bits; the logits are scaled back by 2^e.  Within block c, MMA 0 pairs
+  // k = 2t, 2t+1 with channels 32c + 8t, +1 and k = 2t+8, 2t+9 with 32c + 8t + 2, +3;
+  // MMA 1 the next four channels, so that a thread's codes of a row are one 32-bit word.
+  //   Other warps (sink, window, partial chunk): mma.sync m16n8k8 TF32, exact for the
+  // BF16 rows and query; step j pairs k = t with channel 32c + 8t + 2j and k = t + 4
+  // with the next channel.
+  if (fast) {
+    uint32_t qh[NT][NB][4];
+    float qsc[NT];  // 2^e of head 8n + g
+#pragma unroll
+    for (int n = 0; n < NT; ++n) {
+      const bool hv = 8 * n + g < G;
+      float amax = 0.0f;
+#pragma unroll
+      for (int c = 0; c < NB; ++c)
+#pragma unroll
+        for (int m = 0; m < 8; ++m)
+          amax = fmaxf(amax, hv ? fabsf(qs[(8 * n + g) * D + 32 * c + 8 * tq + m]) : 0.0f);
+      amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+      amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+      const int ex = (int)((__float_as_uint(amax) >> 23) & 0xFFu) - 127;
+      const int e = max(-110, min(110, ex - 14));
+      const float down = pow2f(-e);
+      qsc[n] = pow2f(e);
+#pragma unroll
+      for (int c = 0; c < NB; ++c)
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+          const float x0 = hv ? qs[(8 * n + g) * D + 32 * c + 8 * tq + 2 * m] * down : 0.0f;
+          const float x1 = hv ? qs[(8 * n + g) * D + 32 * c + 8 * tq + 2 * m + 1] * down : 0.0f;
+          const __half2 h2 = __floats2half2_rn(x0, x1);
+          qh[n][c][m] = *reinterpret_cast<const uint32_t*>(&h2);
+        }
+    }
+#pragma unroll
+    for (int tile = 0; tile < 2; ++tile) {
+      const int r_lo = wt0 + 16 * tile + g, r_hi = r_lo + 8;
+      const uint32_t ks_lo = __shfl_sync(0xffffffffu, ksw, 16 * tile + g);
+      const uint32_t ks_hi = __shfl_sync(0xffffffffu, ksw, 16 * tile + g + 8);
+      float s[NT][4];
+#pragma unroll
+      for (int n = 0; n < NT; ++n)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) s[n][e] = 0.0f;
+#pragma unroll
+      for (int c = 0; c < NB; ++c) {
+        const uint32_t kw_lo = *reinterpret_cast<const uint32_t*>(kcs + r_lo * (D / 2) + 16 * c + 4 * tq);
+        const uint32_t kw_hi = *reinterpret_cast<const uint32_t*>(kcs + r_hi * (D / 2) + 16 * c + 4 * tq);
+        uint32_t al[4], ah[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          al[j] = e2m1x2_to_h2((kw_lo >> (8 * j)) & 0xFFu);
+          ah[j] = e2m1x2_to_h2((kw_hi >> (8 * j)) & 0xFFu);
+        }
+        const float sc_lo = e8m0_value((ks_lo >> (8 * c)) & 0xFFu), sc_hi = e8m0_value((ks_hi >> (8 * c)) & 0xFFu);
+#pragma unroll
+        for (int n = 0; n < NT; ++n) {
+          float cb[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+          mma_f16(cb, al[0], ah[0], al[1], ah[1], qh[n][c][0], qh[n][c][1]);
+          mma_f16(cb, al[2], ah[2], al[3], ah[3], qh[n][c][2], qh[n][c][3]);
+          s[n][0] = fmaf(cb[0], sc_lo, s[n][0]);
+          s[n][1] = fmaf(cb[1], sc_lo, s[n][1]);
+          s[n][2] = fmaf(cb[2], sc_hi, s[n][2]);
+          s[n][3] = fmaf(cb[3], sc_hi, s[n][3]);
+        }
+      }
+#pragma unroll
+      for (int n = 0; n < NT; ++n)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int h = 8 * n + 2 * tq + e;
+          const float up = __shfl_sync(0xffffffffu, qsc[n], (2 * tq + e) << 2) * p.scale;
+          if (h < G) {
+            ps[h * kPS + r_lo] = s[n][e] * up;
+            ps[h * kPS + r_hi] = s[n][2 + e] * up;
+          }
+        }
+    }
+  } else {
     float bq[NT][NB][8];
 #pragma unroll
     for (int n = 0; n < NT; ++n)
@@ -305,14 +402,8 @@ __global__ void __launch_bounds__(kThreads, G <= 4 ? 4 : 2) decode_partial_kerne
       const int r_lo = wt0 + 16 * tile + g, r_hi = r_lo + 8;
       const bool v_lo = r_lo < nt, v_hi = r_hi < nt;
       const bool h_lo = v_lo && high(r_lo), h_hi = v_hi && high(r_hi);
-      uint32_t ks_lo = 0x7F7F7F7Fu, ks_hi = 0x7F7F7F7Fu;
-      if (fast) {
-        ks_lo = __shfl_sync(0xffffffffu, ksw, 16 * tile + g);
-        ks_hi = __shfl_sync(0xffffffffu, ksw, 16 * tile + g + 8);
-      } else {
-        if (v_lo && !h_lo) ks_lo = load_scales<D>(p.ksc, row0 + r_lo);
-        if (v_hi && !h_hi) ks_hi = load_scales<D>(p.ksc, row0 + r_hi);
-      }
+      const uint32_t ks_lo = (v_lo && !h_lo) ? load_scales<D>(p.ksc, row0 + r_lo) : 0x7F7F7F7Fu;
+      const uint32_t ks_hi = (v_hi && !h_hi) ? load_scales<D>(p.ksc, row0 + r_hi) : 0x7F7F7F7Fu;
       float s[NT][4];
 #pragma unroll
       for (int n = 0; n < NT; ++n)
@@ -321,22 +412,8 @@ __global__ void __launch_bounds__(kThreads, G <= 4 ? 4 : 2) decode_partial_kerne
 #pragma unroll
       for (int c = 0; c < NB; ++c) {
         float a_lo[8], a_hi[8];
-        if (fast) {
-          const uint32_t kw_lo = *reinterpret_cast<const uint32_t*>(kcs + r_lo * (D / 2) + 16 * c + 4 * tq);
-          const uint32_t kw_hi = *reinterpret_cast<const uint32_t*>(kcs + r_hi * (D / 2) + 16 * c + 4 * tq);
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const float2 xl = e2m1x2_to_float2((kw_lo >> (8 * j)) & 0xFFu);
-            const float2 xh = e2m1x2_to_float2((kw_hi >> (8 * j)) & 0xFFu);
-            a_lo[2 * j] = xl.x;
-            a_lo[2 * j + 1] = xl.y;
-            a_hi[2 * j] = xh.x;
-            a_hi[2 * j + 1] = xh.y;
-          }
-        } else {
-          load_k8<D>(p, row0 + r_lo, v_lo, h_lo, c, tq, a_lo);
-          load_k8<D>(p, row0 + r_hi, v_hi, h_hi, c, tq, a_hi);
-        }
+        load_k8<D>(p, row0 + r_lo, v_lo, h_lo, c, tq, a_lo);
+        load_k8<D>(p, row0 + r_hi, v_hi, h_hi, c, tq, a_hi);
         const float sc_lo = e8m0_value((ks_lo >> (8 * c)) & 0xFFu), sc_hi = e8m0_value((ks_hi >> (8 * c)) & 0xFFu);
 #pragma unroll
         for (int n = 0; n < NT; ++n) {

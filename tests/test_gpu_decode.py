@@ -8,6 +8,8 @@ tokens one at a time equal to quantising the whole cache, and the output
 within max|err| <= 2e-2 * max|O_ref| and relative L2 <= 5e-3 (LSE within
 1e-3) of the oracle on the same seeded inputs.
 """
+import math
+
 import numpy as np
 import pytest
 import torch
@@ -42,8 +44,10 @@ def _check_cache(k, v, cache):
     assert np.array_equal(got["vsc"].reshape(ref["v_sc"].shape), ref["v_sc"]), "V scales"
 
 
-def _run(B, Hq, Hkv, L, d, seed=0, scale=0.0, check_cache=True, batches=None):
+def _run(B, Hq, Hkv, L, d, seed=0, scale=0.0, check_cache=True, batches=None, q_mul=1.0):
     q, k, v = _inputs(B, Hq, Hkv, L, d, seed)
+    if q_mul != 1.0:  # a power of two: the BF16 query is scaled exactly
+        q = (q.float() * q_mul).to(torch.bfloat16)
     qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
     cache = mq.decode_quantize_cache(kd, vd)
     o, lse = mq.decode_step(qd, kd, vd, cache, softmax_scale=scale, want_lse=True)
@@ -97,3 +101,11 @@ def test_decode_cache_is_appendable():
     torch.cuda.synchronize()
     for f in whole:
         assert torch.equal(whole[f], part[f]), f
+
+
+@pytest.mark.parametrize("q_mul,scale", [(2.0 ** -24, 2.0 ** 24), (2.0 ** 12, 2.0 ** -12)])
+def test_decode_query_magnitude_extremes(q_mul, scale):
+    """The logits of quantised tokens run in FP16 with the query rescaled per head by a
+    power of two; a query 2^24 times smaller or 2^12 times larger than usual (softmax
+    scale compensating, so the logits are the usual ones) must still match the oracle."""
+    _run(2, 8, 2, 1024, 128, seed=11, scale=scale / math.sqrt(128), check_cache=False, q_mul=q_mul)
