@@ -24,18 +24,25 @@ __global__ void __launch_bounds__(256) amax_head_kernel(const __nv_bfloat16* __r
   const int bh = blockIdx.y;
   const uint4* p = reinterpret_cast<const uint4*>(x + (long long)bh * per_head);
   const long long nvec = per_head / 8;
+  const long long stride = (long long)gridDim.x * blockDim.x;
   uint32_t m = 0;
-  for (long long v = (long long)blockIdx.x * blockDim.x + threadIdx.x; v < nvec;
-       v += (long long)gridDim.x * blockDim.x) {
-    uint4 u = __ldg(p + v);
-    uint32_t w[4] = {u.x, u.y, u.z, u.w};
+  // |bf16| as float bits: clear the sign, shift into the high half
+  auto fold = [&](const uint4& u) {
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
-    for (int t = 0; t < 4; ++t) {
-      // |bf16| as float bits: clear the sign, shift into the high half
-      uint32_t lo = (w[t] & 0x7FFFu) << 16, hi = w[t] & 0x7FFF0000u;
-      m = max(m, max(lo, hi));
-    }
+    for (int t = 0; t < 4; ++t) m = max(m, max((w[t] & 0x7FFFu) << 16, w[t] & 0x7FFF0000u));
+  };
+  long long v = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  // four independent 16-byte loads in flight per thread
+  for (; v + 3 * stride < nvec; v += 4 * stride) {
+    const uint4 u0 = __ldg(p + v), u1 = __ldg(p + v + stride), u2 = __ldg(p + v + 2 * stride),
+                u3 = __ldg(p + v + 3 * stride);
+    fold(u0);
+    fold(u1);
+    fold(u2);
+    fold(u3);
   }
+  for (; v < nvec; v += stride) fold(__ldg(p + v));
   m = __reduce_max_sync(0xffffffffu, m);
   if ((threadIdx.x & 31) == 0 && m != 0) atomicMax(amax + bh, m);
 }
@@ -56,15 +63,27 @@ __global__ void __launch_bounds__(256) amax_chan_kernel(const __nv_bfloat16* __r
   const int r1 = min(N, r0 + rows_per_block);
   uint32_t m[8] = {0, 0, 0, 0, 0, 0, 0, 0};
   const __nv_bfloat16* base = v + (long long)bh * N * D + g * 8;
-  for (int r = r0 + rr; r < r1; r += RS) {
-    uint4 u = __ldg(reinterpret_cast<const uint4*>(base + (long long)r * D));
-    uint32_t w[4] = {u.x, u.y, u.z, u.w};
+  auto fold = [&](const uint4& u) {
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
     for (int t = 0; t < 4; ++t) {
       m[2 * t] = max(m[2 * t], (w[t] & 0x7FFFu) << 16);
       m[2 * t + 1] = max(m[2 * t + 1], w[t] & 0x7FFF0000u);
     }
+  };
+  int r = r0 + rr;
+  // four independent 16-byte loads in flight per thread
+  for (; r + 3 * RS < r1; r += 4 * RS) {
+    const uint4 u0 = __ldg(reinterpret_cast<const uint4*>(base + (long long)r * D));
+    const uint4 u1 = __ldg(reinterpret_cast<const uint4*>(base + (long long)(r + RS) * D));
+    const uint4 u2 = __ldg(reinterpret_cast<const uint4*>(base + (long long)(r + 2 * RS) * D));
+    const uint4 u3 = __ldg(reinterpret_cast<const uint4*>(base + (long long)(r + 3 * RS) * D));
+    fold(u0);
+    fold(u1);
+    fold(u2);
+    fold(u3);
   }
+  for (; r < r1; r += RS) fold(__ldg(reinterpret_cast<const uint4*>(base + (long long)r * D)));
 #pragma unroll
   for (int t = 0; t < 8; ++t) red[rr][g * 8 + t] = m[t];
   __syncthreads();
@@ -127,12 +146,34 @@ __global__ void __launch_bounds__(256) nvfp4_pack_kernel(
     const float den = __fmul_rn(sd, g);
     uint32_t lo = 0, hi = 0;
     if (sd > 0.0f) {
+      // The code of the correctly rounded quotient x / den, without a division per
+      // element: q = x * fl(1/den) is within 1.5 ulps of it, so q (1 - 2^-20) and
+      // q (1 + 2^-20) bracket it, and the e2m1 rounding (monotone) of the two ends
+      // decides the code when they agree.  Pairs whose ends disagree (a quotient at a
+      // rounding threshold) take the correctly rounded division.  A divisor below
+      // 2^-100 (reciprocal near overflow) takes the division for the whole block.
+      const bool recip_ok = den >= 7.888609052210118e-31f;  // 2^-100
+      const float rcp = __frcp_rn(den);
+      const uint64_t r2 = f2pack(rcp, rcp);
+      const uint64_t dn2 = f2pack(0.99999904632568359375f, 0.99999904632568359375f);  // 1 - 2^-20
+      const uint64_t up2 = f2pack(1.00000095367431640625f, 1.00000095367431640625f);  // 1 + 2^-20
+      uint32_t code[8];
 #pragma unroll
-      for (int e = 0; e < 4; ++e)
-        lo |= cvt_e2m1x2(__fdiv_rn(f[2 * e], den), __fdiv_rn(f[2 * e + 1], den)) << (8 * e);
+      for (int e = 0; e < 8; ++e) {
+        const float fa = f[2 * e], fb = f[2 * e + 1];
+        const uint64_t q2 = fmul2(f2pack(fa, fb), r2);
+        float la, lb, ha, hb;
+        f2unpack(fmul2(q2, dn2), la, lb);
+        f2unpack(fmul2(q2, up2), ha, hb);
+        uint32_t c = cvt_e2m1x2(la, lb);
+        if (!recip_ok || c != cvt_e2m1x2(ha, hb)) c = cvt_e2m1x2(__fdiv_rn(fa, den), __fdiv_rn(fb, den));
+        code[e] = c;
+      }
 #pragma unroll
-      for (int e = 0; e < 4; ++e)
-        hi |= cvt_e2m1x2(__fdiv_rn(f[8 + 2 * e], den), __fdiv_rn(f[9 + 2 * e], den)) << (8 * e);
+      for (int e = 0; e < 4; ++e) {
+        lo |= code[e] << (8 * e);
+        hi |= code[4 + e] << (8 * e);
+      }
     }
     out[2 * b] = lo;
     out[2 * b + 1] = hi;
