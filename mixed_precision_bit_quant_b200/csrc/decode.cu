@@ -135,8 +135,12 @@ __host__ __device__ constexpr int osum_floats(int D, int G) { return (kThreads /
 __host__ __device__ constexpr int kstage_floats(int D) { return kChunk * (D / 2) / 4; }
 __host__ __device__ constexpr int vstage_floats(int D) { return kChunk * D / 4; }
 __host__ __device__ constexpr bool osum_in_kstage(int D, int G) { return osum_floats(D, G) <= kstage_floats(D); }
+// The logits' FP16 query fragments of every lane, built once per CTA: [32 lanes][NT][NB][4]
+// f16x2 words (NT = 8-head tiles, NB = 32-channel blocks), then one exponent per head (16
+// words, keeping what follows 8-byte aligned).
+__host__ __device__ constexpr int qfrag_words(int D, int G) { return 32 * ((G + 7) / 8) * (D / 32) * 4 + 16; }
 __host__ __device__ constexpr int partial_smem_floats(int D, int G) {
-  return kstage_floats(D) + vstage_floats(D) + G * D + G * kPS + 2 * G +
+  return kstage_floats(D) + vstage_floats(D) + qfrag_words(D, G) + G * kPS + 2 * G +
          (osum_in_kstage(D, G) ? 0 : osum_floats(D, G)) + 4 /* mbarrier */;
 }
 
@@ -252,8 +256,9 @@ __global__ void __launch_bounds__(kThreads, G <= 4 ? 4 : 2) decode_partial_kerne
   extern __shared__ __align__(16) float dsm[];
   uint8_t* kcs = reinterpret_cast<uint8_t*>(dsm);                 // [kChunk][D/2] staged K codes
   uint8_t* vcs = kcs + kChunk * (D / 2);                           // [kChunk][D] staged V codes
-  float* qs = dsm + kstage_floats(D) + vstage_floats(D);           // [G][D]
-  float* ps = qs + G * D;                                          // [G][kPS]
+  uint32_t* qfrag = reinterpret_cast<uint32_t*>(dsm + kstage_floats(D) + vstage_floats(D));  // [32][NT][NB][4]
+  int* qexp = reinterpret_cast<int*>(qfrag + 32 * NT * NB * 4);   // [G] per-head exponent e
+  float* ps = dsm + kstage_floats(D) + vstage_floats(D) + qfrag_words(D, G);  // [G][kPS]
   float* red = ps + G * kPS;                                       // [G][2]
   float* osum = osum_in_kstage(D, G) ? dsm : red + 2 * G;          // [8 warps][G][D]
   uint64_t* stage_bar = reinterpret_cast<uint64_t*>(red + 2 * G + (osum_in_kstage(D, G) ? 0 : osum_floats(D, G)));
@@ -269,8 +274,36 @@ __global__ void __launch_bounds__(kThreads, G <= 4 ? 4 : 2) decode_partial_kerne
     bulk_load(smem_u32(kcs), p.kc + row0 * (D / 2), kChunk * (D / 2), bar);
     bulk_load(smem_u32(vcs), p.vc + row0 * D, kChunk * D, bar);
   }
-  for (int i = threadIdx.x; i < G * D; i += kThreads)
-    qs[i] = __bfloat162float(p.q[((long long)b * p.Hq + hk * G + i / D) * D + i % D]);
+  // The group's query: each head's largest |q| (as FP32 bits, which order like the
+  // values), then every lane's FP16 fragments of the logits' products, built once here:
+  // word (l, n, c, m) = q[8n + l/4][32c + 8(l%4) + 2m .. +1] * 2^-e, e per head (below).
+  const __nv_bfloat16* qg = p.q + ((long long)b * p.Hq + hk * G) * D;
+  if (threadIdx.x < G) qexp[threadIdx.x] = 0;
+  __syncthreads();
+  for (int i = threadIdx.x; i < G * D; i += kThreads) {  // a warp's 32 elements are one head's
+    uint32_t m = __float_as_uint(fabsf(__bfloat162float(qg[i])));
+    m = __reduce_max_sync(0xffffffffu, m);
+    if (lane == 0) atomicMax(qexp + i / D, (int)m);
+  }
+  __syncthreads();
+  if (threadIdx.x < G) {
+    // e = floor(log2 amax) - 14 puts the head's largest component in [2^14, 2^15)
+    const int ex = (int)((((uint32_t)qexp[threadIdx.x]) >> 23) & 0xFFu) - 127;
+    qexp[threadIdx.x] = max(-110, min(110, ex - 14));
+  }
+  __syncthreads();
+  for (int wi = threadIdx.x; wi < 32 * NT * NB * 4; wi += kThreads) {
+    const int m = wi & 3, c = (wi >> 2) % NB, n = (wi >> 2) / NB % NT, l = wi / (4 * NB * NT);
+    const int h = 8 * n + (l >> 2), ch = 32 * c + 8 * (l & 3) + 2 * m;
+    uint32_t w = 0u;
+    if (h < G) {
+      const float down = pow2f(-qexp[h]);
+      const __nv_bfloat162 q2 = *reinterpret_cast<const __nv_bfloat162*>(qg + h * D + ch);
+      const __half2 h2 = __floats2half2_rn(__low2float(q2) * down, __high2float(q2) * down);
+      w = *reinterpret_cast<const uint32_t*>(&h2);
+    }
+    qfrag[wi] = w;
+  }
   __syncthreads();
   auto high = [&](int tt) -> bool {
     const int t = t0 + tt;
@@ -319,32 +352,16 @@ __global__ void __launch_bounds__(kThreads, G <= 4 ? 4 : 2) decode_partial_kerne
   // with the next channel.
   if (fast) {
     uint32_t qh[NT][NB][4];
-    float qsc[NT];  // 2^e of head 8n + g
 #pragma unroll
-    for (int n = 0; n < NT; ++n) {
-      const bool hv = 8 * n + g < G;
-      float amax = 0.0f;
+    for (int n = 0; n < NT; ++n)
 #pragma unroll
-      for (int c = 0; c < NB; ++c)
-#pragma unroll
-        for (int m = 0; m < 8; ++m)
-          amax = fmaxf(amax, hv ? fabsf(qs[(8 * n + g) * D + 32 * c + 8 * tq + m]) : 0.0f);
-      amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
-      amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
-      const int ex = (int)((__float_as_uint(amax) >> 23) & 0xFFu) - 127;
-      const int e = max(-110, min(110, ex - 14));
-      const float down = pow2f(-e);
-      qsc[n] = pow2f(e);
-#pragma unroll
-      for (int c = 0; c < NB; ++c)
-#pragma unroll
-        for (int m = 0; m < 4; ++m) {
-          const float x0 = hv ? qs[(8 * n + g) * D + 32 * c + 8 * tq + 2 * m] * down : 0.0f;
-          const float x1 = hv ? qs[(8 * n + g) * D + 32 * c + 8 * tq + 2 * m + 1] * down : 0.0f;
-          const __half2 h2 = __floats2half2_rn(x0, x1);
-          qh[n][c][m] = *reinterpret_cast<const uint32_t*>(&h2);
-        }
-    }
+      for (int c = 0; c < NB; ++c) {
+        const uint4 u = *reinterpret_cast<const uint4*>(qfrag + ((lane * NT + n) * NB + c) * 4);
+        qh[n][c][0] = u.x;
+        qh[n][c][1] = u.y;
+        qh[n][c][2] = u.z;
+        qh[n][c][3] = u.w;
+      }
 #pragma unroll
     for (int tile = 0; tile < 2; ++tile) {
       const int r_lo = wt0 + 16 * tile + g, r_hi = r_lo + 8;
@@ -382,7 +399,7 @@ __global__ void __launch_bounds__(kThreads, G <= 4 ? 4 : 2) decode_partial_kerne
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
           const int h = 8 * n + 2 * tq + e;
-          const float up = __shfl_sync(0xffffffffu, qsc[n], (2 * tq + e) << 2) * p.scale;
+          const float up = (h < G ? pow2f(qexp[h]) : 0.0f) * p.scale;
           if (h < G) {
             ps[h * kPS + r_lo] = s[n][e] * up;
             ps[h * kPS + r_hi] = s[n][2 + e] * up;
@@ -396,7 +413,8 @@ __global__ void __launch_bounds__(kThreads, G <= 4 ? 4 : 2) decode_partial_kerne
 #pragma unroll
       for (int c = 0; c < NB; ++c)
 #pragma unroll
-        for (int m = 0; m < 8; ++m) bq[n][c][m] = (8 * n + g < G) ? qs[(8 * n + g) * D + 32 * c + 8 * tq + m] : 0.0f;
+        for (int m = 0; m < 8; ++m)
+          bq[n][c][m] = (8 * n + g < G) ? __bfloat162float(qg[(8 * n + g) * D + 32 * c + 8 * tq + m]) : 0.0f;
 #pragma unroll
     for (int tile = 0; tile < 2; ++tile) {
       const int r_lo = wt0 + 16 * tile + g, r_hi = r_lo + 8;
