@@ -60,19 +60,6 @@ constexpr int kSoftmaxRegs = 152, kOtherRegs = 56;  // 3*128*152 + 128*56 = 512*
 static_assert(kGroups * 128 * kSoftmaxRegs + 128 * kOtherRegs <= 65536, "register split exceeds the launch budget");
 constexpr int kPRing = 8;                           // P_FULL barriers per group
 constexpr int kMaxW = 128;                          // mask words per query tile (T <= 4096)
-#ifndef THRIFT_POLY_PAIRS
-#define THRIFT_POLY_PAIRS 0x0000u
-#endif
-// Element pairs (bit t of 16, for pair t mod 16 of a row) whose exponential runs on the
-// FMA pipe; the rest run on the MUFU.
-constexpr uint32_t kPolyPairs = THRIFT_POLY_PAIRS;
-#ifndef THRIFT_MAX_PUBLISH_CHUNK
-#define THRIFT_MAX_PUBLISH_CHUNK 0
-#endif
-// How many of a tile's four 32-column exponential chunks a softmax warp finishes before it
-// hands the tile's running maximum to the next group (0: right after computing it).
-constexpr int kMaxPublishChunk = THRIFT_MAX_PUBLISH_CHUNK;
-
 // Operand rings: FP4 tiles use NLO slots of K (e2m1 + scales) and of V^T (e4m3);
 // BF16 tiles use NHI slots of bf16 K and V^T.  Producer and MMA issuer walk the
 // tiles in order and count FP4 and BF16 tiles separately to find slot and phase.
@@ -469,7 +456,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float m_new = fmaxf(m_prev, mloc * sc);
       mbuf[wg * 128 + r] = m_new;
       __syncwarp();
-      if (kMaxPublishChunk == 0 && j + 1 < nj && lane == 0) mbar_arrive(mx_out);
+      if (j + 1 < nj && lane == 0) mbar_arrive(mx_out);
       const float alpha = (m_prev == -INFINITY) ? 0.0f : ex2_approx(m_prev - m_new);  // O rescale
       const float beta = (m_ref == -INFINITY) ? 0.0f : ex2_approx(m_ref - m_new);     // own partial sum
       const uint64_t sc2 = f2pack(sc, sc);
@@ -486,27 +473,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
       }
       // per chunk of 32 columns: exponentials in place (v[c] becomes p * 2^8 in FP32),
-      // then P in the tile's own precision only.  The element pairs that kPolyPairs marks
-      // run on the FMA pipe (polynomial), the others on the MUFU.
+      // then P in the tile's own precision only
 #pragma unroll
       for (int ch = 0; ch < 4; ++ch) {
-        // hand m_j to the next group once this warp's exponentials are far enough along that
-        // the next group's (on the same sub-partition's MUFU) follow rather than overlap them
-        if (kMaxPublishChunk > 0 && ch == kMaxPublishChunk && j + 1 < nj) {
-          __syncwarp();
-          if (lane == 0) mbar_arrive(mx_out);
-        }
 #pragma unroll
         for (int t = 16 * ch; t < 16 * ch + 16; ++t) {
           const uint64_t y2 = ffma2(f2pack(__uint_as_float(v[2 * t]), __uint_as_float(v[2 * t + 1])), sc2, nb2);
-          uint64_t e2;
-          if ((kPolyPairs >> (t & 15)) & 1u) {
-            e2 = exp2_poly_x2(y2);
-          } else {
-            float a0, a1;
-            f2unpack(y2, a0, a1);
-            e2 = f2pack(ex2_approx(a0), ex2_approx(a1));
-          }
+          float a0, a1;
+          f2unpack(y2, a0, a1);
+          const uint64_t e2 = f2pack(ex2_approx(a0), ex2_approx(a1));
           acc[t & 3] = fadd2(acc[t & 3], e2);
           float e0, e1;
           f2unpack(e2, e0, e1);
@@ -530,10 +505,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           tmem_st8(p_base + 32 * (j % 3) + 8 * ch, pe);
         }
-      }
-      if (kMaxPublishChunk >= 4 && j + 1 < nj) {
-        __syncwarp();
-        if (lane == 0) mbar_arrive(mx_out);
       }
       float r0, r1, r2, r3, r4, r5, r6, r7;
       f2unpack(acc[0], r0, r1);

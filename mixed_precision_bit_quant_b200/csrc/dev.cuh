@@ -78,46 +78,11 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Non-blocking test of an mbarrier phase.
-__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
-  return ok != 0;
-}
-
-__device__ __forceinline__ uint64_t globaltimer_ns() {
-  uint64_t t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
-}
 __device__ __forceinline__ uint32_t globaltimer_lo() {
   uint32_t t;
   asm volatile("mov.u32 %0, %%globaltimer_lo;" : "=r"(t));
   return t;
 }
-
-// try_wait with a suspend-time hint: a thread whose phase is not complete yet may be
-// suspended for up to `hint_ns` nanoseconds and is woken when the phase completes, so a
-// waiting warp stops issuing instructions instead of polling.
-__device__ __forceinline__ bool mbar_try_wait_suspend(uint32_t bar, uint32_t parity, uint32_t hint_ns) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok) : "r"(bar), "r"(parity), "r"(hint_ns) : "memory");
-  return ok != 0;
-}
-
-// 0: poll with plain try_wait (measured faster in the attention kernel than sleeping
-// with a suspend-time hint, whose wake-up adds latency to every hand-off)
-#ifndef THRIFT_WAIT_HINT_NS
-#define THRIFT_WAIT_HINT_NS 0
-#endif
 
 // Bounded wait on an mbarrier phase.  Returns false (and never hangs) when
 // the wait exceeds `limit_ns` or when another role raised `*abort` (both are
@@ -128,54 +93,12 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
   // the low 32 bits of the nanosecond timer: differences stay exact for limits below 4.29 s
   const uint32_t t0 = globaltimer_lo();
   for (uint32_t it = 1;; ++it) {
-#if THRIFT_WAIT_HINT_NS > 0
-    if (mbar_try_wait_suspend(bar, parity, THRIFT_WAIT_HINT_NS)) return true;
-#else
+    // plain try_wait polling: measured faster in the attention kernel than sleeping with
+    // a suspend-time hint, and no slower than test_wait spinning
     if (mbar_try_wait(bar, parity)) return true;
-#endif
     if ((it & 63u) == 0u) {
       if (*abort) return false;
       if ((uint64_t)(globaltimer_lo() - t0) > limit_ns) return false;
-    }
-  }
-}
-
-// mbar_wait for a thread that is not on the critical path (a producer running ahead):
-// it sleeps in try_wait between checks instead of polling, leaving its issue slots to
-// the other warps of its sub-partition.
-__device__ __forceinline__ bool mbar_wait_sleep(uint32_t bar, uint32_t parity, volatile int* abort,
-                                                uint64_t limit_ns) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const uint32_t t0 = globaltimer_lo();
-  for (;;) {
-    if (mbar_try_wait_suspend(bar, parity, 20000u)) return true;
-    if (*abort) return false;
-    if ((uint64_t)(globaltimer_lo() - t0) > limit_ns) return false;
-  }
-}
-
-// Monotonic counter in shared memory, published with release and read with acquire
-// semantics (CTA scope).
-__device__ __forceinline__ void st_release_u32(uint32_t addr, uint32_t v) {
-  asm volatile("st.release.cta.shared::cta.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
-}
-__device__ __forceinline__ uint32_t ld_acquire_u32(uint32_t addr) {
-  uint32_t v;
-  asm volatile("ld.acquire.cta.shared::cta.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
-  return v;
-}
-// Bounded wait until the counter at `addr` reaches `target`.  Between polls the
-// thread sleeps briefly, so a waiting warp leaves its issue slots to the warps
-// that compute.
-__device__ __forceinline__ bool count_wait(uint32_t addr, uint32_t target, volatile int* abort, uint64_t limit_ns) {
-  if (ld_acquire_u32(addr) >= target) return true;
-  uint64_t t0 = globaltimer_ns();
-  for (uint32_t it = 1;; ++it) {
-    __nanosleep(20);
-    if (ld_acquire_u32(addr) >= target) return true;
-    if ((it & 63u) == 0u) {
-      if (*abort) return false;
-      if (globaltimer_ns() - t0 > limit_ns) return false;
     }
   }
 }
@@ -239,12 +162,6 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint3
   d |= (uint64_t)1 << 46;
   d |= (uint64_t)(swz & 7u) << 61;
   return d;
-}
-
-// The descriptor of start address 0: add (address >> 4) for a tile (addresses below 256 KB).
-__host__ __device__ constexpr uint64_t smem_desc_tmpl(uint32_t lbo, uint32_t sbo, uint32_t swz) {
-  return (uint64_t)((lbo >> 4) & 0x3FFFu) << 16 | (uint64_t)((sbo >> 4) & 0x3FFFu) << 32 | (uint64_t)1 << 46 |
-         (uint64_t)(swz & 7u) << 61;
 }
 
 // Instruction descriptors (M = 128, FP32 accumulate, both operands K-major).
@@ -336,14 +253,6 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
         "r"(r[29]), "r"(r[30]), "r"(r[31])
       : "memory");
 }
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
-      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
-      : "r"(taddr));
-}
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
@@ -357,15 +266,6 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
       : "memory");
 }
 
-// Producer side of a named barrier: arrive without waiting.
-__device__ __forceinline__ void named_bar_arrive(uint32_t id, uint32_t count) {
-  asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(count) : "memory");
-}
-
-__device__ __forceinline__ void tmem_st4(uint32_t taddr, const uint32_t (&r)[4]) {
-  asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1,%2,%3,%4};"
-               ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]) : "memory");
-}
 __device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) {
   asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};"
                ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]),
@@ -404,19 +304,9 @@ __device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
   asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
   return d;
 }
-__device__ __forceinline__ uint64_t fadd2_rm(uint64_t a, uint64_t b) {
-  uint64_t d;
-  asm("add.rm.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-  return d;
-}
 __device__ __forceinline__ uint64_t fmul2(uint64_t a, uint64_t b) {
   uint64_t d;
   asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-  return d;
-}
-__device__ __forceinline__ uint64_t fsub2(uint64_t a, uint64_t b) {
-  uint64_t d;
-  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
   return d;
 }
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
@@ -453,35 +343,6 @@ __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
-}
-
-// 2^y for two lanes on the FMA pipe instead of the MUFU: y = j + f with
-// j = round(y) (adding 1.5 * 2^23 leaves round(y) in the low mantissa bits)
-// and f in [-1/2, 1/2]; 2^f from a degree-4 polynomial whose coefficients
-// minimise the relative error on that interval (Remez exchange, max relative
-// error 2.6e-6 in FP32); 2^j enters by adding j to the exponent field.
-// y is clamped to -126 first, so any finite or -inf input gives a finite
-// result (2^-126 or a value of that size for the clamped inputs).
-__device__ __forceinline__ uint64_t exp2_poly_x2(uint64_t y2) {
-  float y0, y1;
-  f2unpack(y2, y0, y1);
-  const uint64_t y = f2pack(fmaxf(y0, -126.0f), fmaxf(y1, -126.0f));
-  const uint64_t magic = f2pack(12582912.0f, 12582912.0f);
-  const uint64_t t = fadd2(y, magic);          // 1.5 * 2^23 + round(y), exact
-  const uint64_t f = fsub2(y, fsub2(t, magic));  // y - round(y), exact
-  uint64_t p = f2pack(9.570102207362652e-03f, 9.570102207362652e-03f);
-  p = ffma2(p, f, f2pack(5.591785907745361e-02f, 5.591785907745361e-02f));
-  p = ffma2(p, f, f2pack(2.402474433183670e-01f, 2.402474433183670e-01f));
-  p = ffma2(p, f, f2pack(6.931217908859253e-01f, 6.931217908859253e-01f));
-  p = ffma2(p, f, f2pack(9.999992847442627e-01f, 9.999992847442627e-01f));
-  float p0, p1, t0, t1;
-  f2unpack(p, p0, p1);
-  f2unpack(t, t0, t1);
-  // the low 9 bits of t's encoding hold round(y) (two's complement), so
-  // shifting them into the exponent field adds round(y) to p's exponent
-  const float r0 = __uint_as_float(__float_as_uint(p0) + (__float_as_uint(t0) << 23));
-  const float r1 = __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23));
-  return f2pack(r0, r1);
 }
 
 }  // namespace thrift
