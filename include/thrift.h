@@ -77,7 +77,8 @@ typedef struct {
  *
  * FP8 V: per (batch, kv head, channel c) the smallest integer e_c with
  * amax_c <= 448 * 2^e_c (0 for a zero channel); v_code = e4m3(v * 2^-e_c)
- * and the exact BF16 copy v * 2^-e_c, both stored transposed (channel-major)
+ * and the BF16 copy v * 2^-e_c (exact; values that fall into the BF16
+ * subnormals round to nearest even), both stored transposed (channel-major)
  * and zero-padded to Np keys.
  */
 typedef struct {

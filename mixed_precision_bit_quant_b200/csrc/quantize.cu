@@ -187,7 +187,7 @@ __global__ void __launch_bounds__(256) nvfp4_pack_kernel(
 }
 
 // ---------------------------------------------------------------------------
-// FP8 V: per-channel exponent, e4m3 codes and exact BF16 copy, both
+// FP8 V: per-channel exponent, e4m3 codes and BF16 copy, both
 // transposed to [BH][D][Np].  grid (T, BH); a 128-key tile per block.
 // ---------------------------------------------------------------------------
 template <int D>
@@ -233,9 +233,11 @@ __global__ void __launch_bounds__(256) fp8_v_pack_kernel(
 #pragma unroll
     for (int k = 0; k < 16; ++k) {
       const float x = __bfloat162float(tile[seg * 16 + k][c]);
-      const float y = __fmul_rn(x, sc);  // exact: power of two
+      const float y = __fmul_rn(x, sc);  // exact (a power of two) unless far in the subnormals
       codes[k >> 2] |= e4m3_code(y) << (8 * (k & 3));
-      const uint32_t yb = __float_as_uint(y) >> 16;  // exact in bf16
+      // the BF16 copy: exact for every y >= 2^-126 (8 significant bits); BF16 subnormals
+      // round to nearest, ties to even
+      const uint32_t yb = __bfloat16_as_ushort(__float2bfloat16_rn(y));
       if (k & 1) bf[k >> 1] |= yb << 16; else bf[k >> 1] = yb;
     }
     const long long off = ((long long)bh * D + c) * Np + n0 + seg * 16;

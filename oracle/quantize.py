@@ -20,8 +20,10 @@ NVFP4 one is written out, in FP32 with correctly rounded IEEE operations
 
 V is quantised to e4m3 with one power-of-two scale per (batch, kv head,
 channel): ``e_c`` is the smallest integer with ``amax_c <= 448 * 2**e_c``
-(0 for an all-zero channel); ``v_code = e4m3(v * 2**-e_c)`` and the exact
-BF16 copy ``v_s = v * 2**-e_c`` feeds the BF16 tiles.
+(0 for an all-zero channel); ``v_code = e4m3(v * 2**-e_c)`` and the BF16
+copy ``v_s = v * 2**-e_c`` feeds the BF16 tiles -- exact, except for values
+that fall into the BF16 subnormals (a channel whose maximum is 2**134 or more
+times larger), which round to nearest with ties to even.
 
 Parity pins: tests/test_oracle_quantize.py (bound on the dequantisation
 error, the block maximum lands on +-6, exact V rescaling, minimal e_c,
@@ -110,9 +112,15 @@ def fp8_v_quantize(v):
     B, H, N, d = v.shape
     amax = np.abs(v).max(axis=2) if N > 0 else np.zeros((B, H, d), F32)
     e = v_channel_exponent(amax)
-    scaled = np.ldexp(v, (-e)[:, :, None, :].astype(np.int32)).astype(F32)   # exact
+    # v * 2**-e_c in FP32: exact unless it falls below 2**-142, deep in the subnormals
+    scaled = np.ldexp(v.astype(np.float64), (-e)[:, :, None, :].astype(np.int32)).astype(F32)
     v_code = e4m3_encode(scaled)
-    return v_code, e.astype(np.int8), scaled
+    # the BF16 copy: exact wherever v * 2**-e_c is a BF16 value, which every value at or
+    # above 2**-126 is (8 significant bits); below, in the BF16 subnormals, round to
+    # nearest, ties to even, sign kept (a value below 2**-142 rounds to +-0 either way,
+    # so the FP32 rounding above cannot change the result)
+    v_s = torch.from_numpy(np.ascontiguousarray(scaled)).to(torch.bfloat16).float().numpy()
+    return v_code, e.astype(np.int8), v_s
 
 
 def quantize(q, k, v):

@@ -126,3 +126,30 @@ def test_nibble_packing_roundtrip(rng):
     p = pack_nibbles(c)
     assert p[0, 0] == (c[0, 0] | (c[0, 1] << 4))
     assert np.array_equal(unpack_nibbles(p), c)
+
+
+def test_v_copy_rounds_bf16_subnormals_to_nearest_even():
+    """A channel whose maximum is far above its other values: v * 2**-e_c falls into the
+    BF16 subnormals (spacing 2**-133), where the copy rounds to the nearest grid point
+    with ties to even and keeps the sign; the e4m3 codes of those values are +-0."""
+    amax = 2.0 ** 127                     # e_c = 119: 2**127 <= 448 * 2**119
+    tiny = np.array([0.25, 0.375, 0.5, 0.75, 1.0, 1.25, 1.5, 2.5, 3.0, 100.0], dtype=np.float64)
+    vals = np.concatenate([[amax], tiny * 2.0 ** -14, -tiny * 2.0 ** -14])  # all BF16 values
+    v = torch.tensor(vals, dtype=torch.float32).to(torch.bfloat16).reshape(1, 1, -1, 1)
+    assert np.array_equal(v.double().numpy().ravel(), vals)
+    v_code, v_exp, v_s = fp8_v_quantize(v)
+    assert int(v_exp[0, 0, 0]) == 119
+    exact = vals * 2.0 ** -119            # the tiny ones: 0.25 .. 100 times 2**-133
+    step = 2.0 ** -133
+    # brute-force nearest grid point, ties to the even multiple
+    k = np.floor(np.abs(exact) / step)
+    frac = np.abs(exact) / step - k
+    up = (frac > 0.5) | ((frac == 0.5) & (k % 2 == 1))
+    want = np.sign(exact) * (k + up) * step
+    got = v_s.astype(np.float64).ravel()
+    assert np.array_equal(got[1:], want[1:])
+    assert np.array_equal(np.signbit(got[1:]), np.signbit(exact[1:]))   # -0 kept
+    assert got[0] == 256.0
+    # the e4m3 codes of the tiny values are zeros with their signs
+    codes = v_code.ravel()[1:]
+    assert np.array_equal(codes, np.where(exact[1:] < 0, 0x80, 0x00))
