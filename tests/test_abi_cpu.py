@@ -108,3 +108,64 @@ def test_maximum_sizes_on_host():
     assert L.thrift_quant_bytes(ctypes.byref(wide), 0) == 0
     ok = mq.make_shape(1, 32767, 32767, 128, 64, False)
     assert L.thrift_quant_bytes(ctypes.byref(ok), 0) == 32767 * 128 * 32
+
+
+def _dshape(B=2, Hq=8, Hkv=2, L=1000, d=128, scale=0.0):
+    return _lib.DecodeShape(B, Hq, Hkv, L, d, scale)
+
+
+def test_decode_cache_and_workspace_sizes():
+    L = mq.lib()
+    s = _dshape()
+    rows = 2 * 2 * 1000
+    want = [rows * 64, rows * 4, rows * 128, rows * 4]   # e2m1 K, e8m0 K scales, e4m3 V, e8m0 V scales
+    assert [L.thrift_decode_cache_bytes(ctypes.byref(s), f) for f in range(4)] == want
+    assert L.thrift_decode_cache_bytes(ctypes.byref(s), 4) == 0
+    # one softmax state (max, sum, O[d]) per query head and 256-token chunk
+    assert L.thrift_decode_workspace_bytes(ctypes.byref(s)) == 4 * 2 * 8 * 4 * (2 + 128)
+    s64 = _dshape(B=1, Hq=4, Hkv=4, L=256, d=64)
+    assert L.thrift_decode_cache_bytes(ctypes.byref(s64), 1) == 256 * 4 * 2
+    assert L.thrift_decode_workspace_bytes(ctypes.byref(s64)) == 4 * 4 * 1 * (2 + 64)
+
+
+@pytest.mark.parametrize("bad,status", [
+    (dict(d=96), _lib.THRIFT_ERR_UNSUPPORTED),
+    (dict(Hq=6, Hkv=2), _lib.THRIFT_ERR_UNSUPPORTED),      # group of 3 heads
+    (dict(Hq=64, Hkv=2), _lib.THRIFT_ERR_UNSUPPORTED),     # group of 32 heads
+    (dict(B=70000, Hq=1, Hkv=1), _lib.THRIFT_ERR_UNSUPPORTED),  # B * Hkv on one grid axis
+    (dict(L=0), _lib.THRIFT_ERR_INVALID),
+    (dict(Hq=6, Hkv=4), _lib.THRIFT_ERR_INVALID),
+    (dict(scale=-1.0), _lib.THRIFT_ERR_INVALID),
+    (dict(scale=float("inf")), _lib.THRIFT_ERR_INVALID),
+])
+def test_decode_shapes_rejected_on_host(bad, status):
+    L = mq.lib()
+    s = _dshape(**bad)
+    assert L.thrift_decode_cache_bytes(ctypes.byref(s), 0) == 0
+    assert L.thrift_decode_workspace_bytes(ctypes.byref(s)) == 0
+    c = _lib.DecodeCacheStruct(16, 16, 16, 16)
+    assert L.thrift_decode_step(ctypes.byref(s), 16, 16, 16, ctypes.byref(c), 16, None, 16, 1 << 30, None) == status
+    assert L.thrift_decode_quantize_cache(ctypes.byref(s), 16, 16, ctypes.byref(c), 0, 1, None) == status
+
+
+def test_decode_pointers_ranges_and_workspace_checked_on_host():
+    L = mq.lib()
+    s = _dshape()
+    ws = L.thrift_decode_workspace_bytes(ctypes.byref(s))
+    c = _lib.DecodeCacheStruct(16, 16, 16, 16)
+    bad_c = _lib.DecodeCacheStruct(16, None, 16, 16)
+    mis_c = _lib.DecodeCacheStruct(16, 16, 24, 16)
+    step = lambda q=16, k=16, v=16, cache=c, o=16, lse=None, w=16, nb=ws: L.thrift_decode_step(  # noqa: E731
+        ctypes.byref(s), q, k, v, ctypes.byref(cache), o, lse, w, nb, None)
+    for kw in (dict(q=None), dict(q=24), dict(k=8), dict(o=None), dict(w=None), dict(cache=bad_c),
+               dict(cache=mis_c), dict(lse=18), dict(nb=ws - 1)):
+        assert step(**kw) == _lib.THRIFT_ERR_INVALID, kw
+    assert L.thrift_decode_step(ctypes.byref(s), 16, 16, 16, None, 16, None, 16, ws, None) == _lib.THRIFT_ERR_INVALID
+    quant = lambda t0, t1, k=16: L.thrift_decode_quantize_cache(  # noqa: E731
+        ctypes.byref(s), k, 16, ctypes.byref(c), t0, t1, None)
+    for t0, t1 in ((-1, 5), (0, 1001), (7, 6)):
+        assert quant(t0, t1) == _lib.THRIFT_ERR_INVALID, (t0, t1)
+    assert quant(0, 5, k=None) == _lib.THRIFT_ERR_INVALID
+    # an empty range is valid and enqueues nothing (no device access)
+    assert quant(5, 5) == _lib.THRIFT_OK
+    assert quant(1000, 1000) == _lib.THRIFT_OK
