@@ -108,3 +108,59 @@ def test_benchmark_and_test_call_patterns_pass_every_check(any_device, name, mon
     qb, kb, vb, ob = (torch.empty_like(t) for t in (q, k, v, o))
     mq.quantize(qb, kb, vb, w.causal, out=quant, ws=ws_q)
     mq.attn_fwd(qb, kb, quant, mask, w.causal, o=ob)
+
+
+def _decode_inputs(B=2, Hq=8, Hkv=2, L=300, d=64):
+    g = torch.Generator().manual_seed(5)
+    q = torch.randn((B, Hq, d), generator=g).to(torch.bfloat16)
+    k = torch.randn((B, Hkv, L, d), generator=g).to(torch.bfloat16)
+    v = torch.randn((B, Hkv, L, d), generator=g).to(torch.bfloat16)
+    return q, k, v
+
+
+def _host_cache(k):
+    B, Hkv, L, d = k.shape
+    rows = B * Hkv * L
+    sizes = dict(kc=rows * d // 2, ksc=rows * d // 32, vc=rows * d, vsc=rows * d // 32)
+    return {f: torch.zeros(n, dtype=torch.uint8) for f, n in sizes.items()}
+
+
+def test_decode_host_tensors_are_refused():
+    q, k, v = _decode_inputs()
+    with pytest.raises(ValueError, match="CUDA"):
+        mq.decode_quantize_cache(k, v)
+    with pytest.raises(ValueError, match="CUDA"):
+        mq.decode_step(q, k, v, _host_cache(k))
+
+
+@pytest.mark.parametrize("bad", ["k_dtype", "v_shape", "q_rank", "q_batch", "q_dim", "cache_small",
+                                 "cache_dtype", "o_dtype", "lse_shape", "strided_v"])
+def test_decode_bad_arguments_are_refused(any_device, bad):
+    q, k, v = _decode_inputs()
+    cache = _host_cache(k)
+    kw = {}
+    match = {"k_dtype": "dtype", "v_shape": "shape", "q_rank": "tensor", "q_batch": "shape", "q_dim": "shape",
+             "cache_small": "too small", "cache_dtype": "dtype", "o_dtype": "dtype", "lse_shape": "shape",
+             "strided_v": "contiguous"}[bad]
+    if bad == "k_dtype":
+        k = k.float()
+    elif bad == "v_shape":
+        v = v[:, :, :-1]
+    elif bad == "q_rank":
+        q = q[0]
+    elif bad == "q_batch":
+        q = q[:1]
+    elif bad == "q_dim":
+        q = torch.zeros((2, 8, 128), dtype=torch.bfloat16)
+    elif bad == "cache_small":
+        cache["vc"] = cache["vc"][:-1]
+    elif bad == "cache_dtype":
+        cache["ksc"] = cache["ksc"].to(torch.int32)
+    elif bad == "o_dtype":
+        kw["o"] = torch.empty(q.shape, dtype=torch.float32)
+    elif bad == "lse_shape":
+        kw["lse"] = torch.empty((2, 7), dtype=torch.float32)
+    else:
+        v = v.transpose(2, 3).contiguous().transpose(2, 3)
+    with pytest.raises(ValueError, match=match):
+        mq.decode_step(q, k, v, cache, **kw)
